@@ -1,0 +1,467 @@
+"""Benchmark of causal kernelized linear attention (phi(x) = x x^T) on B200.
+
+Headline (``value``): chunked-prefill tokens/s on the prefill workload
+B=4, H=8, T=2048, d=32, bf16, chunk 64 -- one step is one kata_prefill call
+over that batch (feature map, intra-chunk contraction, state accumulation,
+carry and readout). The same JSON line carries the decode step (B=64, H=16,
+d=64 from a 4096-token prefix), the long prefill (B=2, H=16, T=16384, d=64)
+and the LoLA schedule (B=2, H=8, T=8192, d=64) as sub-results, the roofline
+of the dominant kernel, the fp64 oracle timed on the host cores, and an
+end-to-end number through the C ABI with host buffers.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kata|reference]
+
+With N > 1 it runs under torchrun, one rank per GPU; every rank runs the same
+per-GPU workload (weak scaling, no collective on the data path) and the
+slowest rank's device time sets the aggregate.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from kernelized_linear_attention_chunked_b200.inputs import (  # noqa: E402
+    WORKLOADS, decode_inputs, prefill_inputs, recall_inputs)
+
+METRIC = "prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s (% HBM BW), 1×B200"
+HEADLINE = "prefill_b4_h8_t2048_d32"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def prefill_flops(w) -> float:
+    """Algorithmic flops of one prefill over the workload: per head-token
+    4 D (d+1) for the inter-chunk readout and state update, and
+    (C+1)(2d+1) for the causal intra-chunk part (half of the square)."""
+    D = w.d * (w.d + 1) // 2
+    per = 4 * D * (w.d + 1) + (w.chunk + 1) * (2 * w.d + 1)
+    return float(per) * w.B * w.H * w.T
+
+
+def prefill_bytes(w) -> float:
+    """Compulsory HBM bytes: q, k, v in, o (fp32) out."""
+    es = 2 if w.dtype == "bf16" else 4
+    return float(w.B * w.H * w.T * w.d * (3 * es + 4))
+
+
+def decode_bytes(w) -> float:
+    """Per step: the fp32 state read and written once, q, k, v in, o out."""
+    D = w.d * (w.d + 1) // 2
+    return float(w.B * w.H * (2 * D * (w.d + 1) * 4 + 3 * w.d * 2 + w.d * 4))
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        return json.loads(p.read_text()), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [x for x in sm if mx and x > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_record(kernel: str, workload: str):
+    """ncu dram bytes per launch recorded under profiles/, if the kernel source
+    has not changed since the counters were taken (else None)."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    rec = json.loads(p.read_text()).get(f"{kernel}@{workload}")
+    if not rec:
+        return None
+    src = ROOT / "kernelized_linear_attention_chunked_b200" / "csrc" / rec["source"]
+    if not src.exists() or hashlib.sha256(src.read_bytes()).hexdigest()[:16] != rec["sha"]:
+        return None
+    return rec["bytes_per_launch"]
+
+
+# ---------------------------------------------------------------- oracle ----
+
+def cpu_baseline(w, max_heads: int | None = None):
+    """The fp64 oracle (recurrent form, the fastest exact CPU form) on a
+    bounded sample of the workload, scaled to tokens/s."""
+    import oracle
+    q, k, v = prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed, recipe=w.recipe)
+    nh = w.B * w.H if max_heads is None else min(max_heads, w.B * w.H)
+    qf, kf, vf = (x.reshape(w.B * w.H, w.T, w.d)[:nh] for x in (q, k, v))
+    t0 = time.perf_counter()
+    oracle.recurrent(qf, kf, vf, w.eps)
+    dt = time.perf_counter() - t0
+    tokens = w.T * nh / w.H  # a token is one position of one sequence (all heads)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"recurrent fp64 form over {nh} of {w.B * w.H} heads x {w.T} tokens "
+                      f"({dt:.2f} s)", "seconds": dt}
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    import oracle  # noqa: F401
+    w = WORKLOADS[HEADLINE]
+    nh = 4  # a bounded sample per step: 4 of 32 heads (about a second of CPU work)
+    for _ in range(args.warmup):
+        cpu_baseline(w, max_heads=nh)
+    times, vals = [], []
+    for _ in range(args.steps):
+        r = cpu_baseline(w, max_heads=nh)
+        times.append(r["seconds"])
+        vals.append(r["value"])
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * float(np.mean(times)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": HEADLINE, "global_batch": w.B, "seq_len": w.T, "heads": w.H,
+                       "head_dim": w.d, "chunk": w.chunk, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle",
+                             "cores": r["cores"], "sample": r["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU ----
+
+def time_events(fn, iters: int, stream) -> float:
+    """Device milliseconds for `iters` calls of fn, CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(iters):
+        fn(i)
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def per_launch_ms(fn, iters: int, stream) -> float:
+    """Mean duration of single calls, each bracketed by its own events."""
+    ts = []
+    for i in range(iters):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn(i)
+        e.record(stream)
+        e.synchronize()
+        ts.append(s.elapsed_time(e))
+    return float(np.mean(ts))
+
+
+def barrier(dist_on):
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, dist_on) -> float:
+    if not dist_on:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_kata(args, rank: int, world: int, dist_on: bool):
+    import kernelized_linear_attention_chunked_b200 as kata
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = load_peaks()
+    w = WORKLOADS[HEADLINE]
+
+    # Headline: prefill over resident inputs. The batch's inputs and outputs
+    # are 21 MB, so R copies rotate (R x 21 MB > L2) and no step finds its
+    # inputs in L2.
+    q, k, v = prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed, recipe=w.recipe)
+    R = int(np.ceil(2 * L2_BYTES / prefill_bytes(w)))
+    sets = [tuple(x.to(dev) for x in (q, k, v)) for _ in range(R)]
+    outs = [torch.empty(w.B, w.H, w.T, w.d, device=dev) for _ in range(R)]
+    ws = torch.empty(max(kata.prefill_workspace_bytes(w.B, w.H, w.T, w.d, w.chunk,
+                                                      torch.bfloat16), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        qq, kk, vv = sets[i % R]
+        kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, state=False, o=outs[i % R],
+                     workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    kata.sync_status()
+    barrier(dist_on)
+    n0 = kata.launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0 = time.perf_counter()
+        ms = time_events(step, args.steps, stream)
+        barrier(dist_on)
+        wall = time.perf_counter() - t0
+    launches = kata.launch_count() - n0
+    kata.sync_status()
+    ms = max_over_ranks(ms, dist_on)
+    tokens_per_step = w.B * w.T
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    ms_step = ms / args.steps
+    flops = prefill_flops(w)
+    tflops = flops / (ms_step / 1e3) / 1e12
+
+    # roofline of the dominant kernel: the prefill kernel, one launch per call
+    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    path = "tc" if kata.prefill_uses_tensor_cores(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16) \
+        else "simt"
+    if path == "tc":
+        roof = {"bound": "tensor", "achieved": flops / (lat / 1e3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        kernel = "prefill_tc_kernel"
+    else:
+        # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x max SM clock
+        alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": flops / (lat / 1e3) / 1e12, "peak": alu_peak,
+                "unit": "TFLOP/s"}
+        kernel = "prefill_simt_kernel"
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
+        else "fallback"
+    roof["kernel"] = kernel
+    roof["launch_ms"] = lat
+    roof["traffic"] = traffic_record(kernel, HEADLINE)
+    roof["algorithmic_bytes"] = prefill_bytes(w)
+    roof["hbm_frac"] = prefill_bytes(w) / (lat / 1e3) / 1e9 / peaks["hbm_gbs"]
+
+    # end to end: host q, k, v in, host o out, through the C ABI
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(w.B, w.H, w.T, w.d).pin_memory()
+    wsh = torch.empty(kata.prefill_host_workspace_bytes(w.B, w.H, w.T, w.d, w.chunk,
+                                                        torch.bfloat16),
+                      dtype=torch.uint8, device=dev)
+
+    def e2e_step(i):
+        kata.prefill_host(qh, kh, vh, w.chunk, w.eps, oh, wsh)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier(dist_on)
+    ms_e2e = max_over_ranks(time_events(e2e_step, args.steps, stream), dist_on)
+    e2e = {"value": world * tokens_per_step * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+           "d2h_bytes_per_step": oh.numel() * 4}
+    del sets, outs, qh, kh, vh, oh, wsh
+
+    sub = {}
+    if not args.headline_only:
+        sub["decode"] = bench_decode(kata, args, dev, stream, peaks, dist_on, world)
+        sub["long_prefill"] = bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world)
+        sub["lola"] = bench_lola(kata, args, dev, stream, dist_on, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, max_heads=8)
+        cpu.pop("seconds")
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": HEADLINE, "global_batch": w.B * world, "seq_len": w.T,
+                       "heads": w.H, "head_dim": w.d, "packed_dim": w.D, "chunk": w.chunk,
+                       "parallelism": f"dp{world}", "path": path,
+                       "l2": f"{R} rotating input sets ({R * prefill_bytes(w) / 2**20:.0f} MB "
+                             "> 126 MB L2)"},
+            "prefill": {"tflops": tflops, "frac_bf16_peak": tflops / peaks["bf16_tflops"],
+                        "peak_source": peak_kind},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clocks.summary(), "wall_s": wall}
+    line.update(sub)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
+    w = WORKLOADS["decode_b64_h16_d64"]
+    kp, vp, q, k, v = decode_inputs(w.B, w.H, w.d, w.prefix, w.steps, dtype=w.dtype, seed=w.seed)
+    D = w.D
+    Hst = torch.zeros(w.B, w.H, D, w.d, device=dev)
+    s = torch.zeros(w.B, w.H, D, device=dev)
+    # the prefix state: the 4096 prefix tokens written in by decode steps
+    # (outputs discarded); not timed
+    kpd = kp.to(dev).permute(2, 0, 1, 3).contiguous()
+    vpd = vp.to(dev).permute(2, 0, 1, 3).contiguous()
+    o = torch.empty(w.B, w.H, w.d, device=dev)
+    for t in range(w.prefix):
+        kata.decode_step(kpd[t], kpd[t], vpd[t], Hst, s, eps=w.eps, o=o)
+    del kpd, vpd
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    nsteps = w.steps
+
+    def step(i):
+        kata.decode_step(qd[i % nsteps], kd[i % nsteps], vd[i % nsteps], Hst, s, eps=w.eps, o=o)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier(dist_on)
+    n0 = kata.launch_count()
+    ms = max_over_ranks(time_events(step, nsteps, stream), dist_on)
+    launches = kata.launch_count() - n0
+    kata.sync_status()
+    ms_step = ms / nsteps
+    gbs = decode_bytes(w) / (ms_step / 1e3) / 1e9
+    return {"workload": w.name, "tokens_per_s": world * w.B * nsteps / (ms / 1e3),
+            "us_per_step": 1e3 * ms_step, "steps": nsteps, "gbs": gbs,
+            "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_step": decode_bytes(w),
+            "gpu_launches": launches, "l2": "state 554 MB > 126 MB L2"}
+
+
+def bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world):
+    w = WORKLOADS["long_prefill_b2_h16_t16384_d64"]
+    q, k, v = (x.to(dev) for x in prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype,
+                                                  seed=w.seed, recipe=w.recipe))
+    o = torch.empty(w.B, w.H, w.T, w.d, device=dev)
+    ws = torch.empty(max(kata.prefill_workspace_bytes(w.B, w.H, w.T, w.d, w.chunk,
+                                                      torch.bfloat16), 1),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        kata.prefill(q, k, v, chunk=w.chunk, eps=w.eps, state=False, o=o, workspace=ws)
+
+    step(0)
+    barrier(dist_on)
+    n = max(2, min(args.steps, 10))
+    ms = max_over_ranks(time_events(step, n, stream), dist_on) / n
+    kata.sync_status()
+    fl = prefill_flops(w)
+    return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
+            "tflops": fl / (ms / 1e3) / 1e12, "frac_bf16_peak": fl / (ms / 1e3) / 1e12 /
+            peaks["bf16_tflops"], "l2": "inputs 335 MB > 126 MB L2"}
+
+
+def bench_lola(kata, args, dev, stream, dist_on, world):
+    w = WORKLOADS["lola_b2_h8_t8192_d64"]
+    q, k, v = (x.to(dev) for x in recall_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed))
+    D = w.D
+    Hst = torch.zeros(w.B, w.H, D, w.d, device=dev)
+    s = torch.zeros_like(Hst[..., 0])
+    o = torch.empty(w.B, w.H, w.T, w.d, device=dev)
+    ws = torch.empty(kata.lola_prefill_workspace_bytes(w.B, w.H, w.T, w.d, w.window, w.cache),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i):
+        Hst.zero_()
+        s.zero_()
+        kata.lola_prefill(q, k, v, window=w.window, cache=w.cache, eps=w.eps, Hst=Hst, s=s,
+                          o=o, workspace=ws)
+
+    step(0)
+    barrier(dist_on)
+    n0 = kata.launch_count()
+    n = 3
+    ms = max_over_ranks(time_events(step, n, stream), dist_on) / n
+    launches = (kata.launch_count() - n0) // n
+    kata.sync_status()
+    return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
+            "updates": w.T // w.window - 1, "gpu_launches_per_pass": launches,
+            "note": "includes two state zero-fills per pass (torch memset)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kata", "reference"], default="kata")
+    ap.add_argument("--headline-only", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist_on = world > 1
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        run_kata(args, rank, world, dist_on)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

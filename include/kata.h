@@ -1,0 +1,234 @@
+/*
+ * kata.h -- C ABI of libkata.so: causal kernelized linear attention with the
+ * rank-one PSD feature phi(x) = x x^T, and the LoLA self-recall-error sparse
+ * cache, on NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, section):
+ *   [KATA] "Kernelized Linear Attention: Breaking the Capacity Wall with
+ *          Symmetric Cones": s1 (fixed-size recurrent state, constant-time
+ *          recurrent inference), s2.1 (the normalising denominator is a
+ *          parameter-free convex output gate), s2.2 (psi(u) = u u^T, whose
+ *          inner products are squared raw inner products), s2.3 (chunked
+ *          parallelism: tensor cores inside a chunk, state propagated across
+ *          chunks; the chunked state form is exact).
+ *   [LoLA] "LoLA: Low-Rank Linear Attention with Sparse Caching":
+ *          Methodology 1-3 (sliding window, recurrent state H_t with
+ *          normaliser s_t, sparse global cache), "Self-Recall Error",
+ *          "Inference strategy" steps 1-4.
+ *
+ * Conventions shared by every entry point
+ *   - Shapes are row-major (C order). B = batch, H = heads, T = tokens,
+ *     d = head dimension (keys, queries and values all have d columns),
+ *     D = d(d+1)/2 = packed feature dimension.
+ *   - Packed state layout (the checkpoint format): phi(x) is the upper
+ *     triangle of x x^T, row (a) major; entry (a, b), a <= b, sits at index
+ *     a*d - a(a-1)/2 + (b - a) and carries a factor sqrt(2) when a < b, so
+ *     that <phi(x), phi(y)> = (x.y)^2 exactly. The state is
+ *     H [B, H, D, d] fp32 = sum_j phi(k_j) v_j^T and s [B, H, D] fp32 =
+ *     sum_j phi(k_j).
+ *   - Causality is inclusive: output i sees tokens j <= i. eps is added to
+ *     every denominator.
+ *   - Pointers named *_dev (and every pointer unless stated) are device
+ *     pointers; *_host pointers are host pointers (pinned memory gives
+ *     asynchronous copies). The caller owns every buffer; the library never
+ *     allocates or frees memory and never synchronises the stream, except
+ *     kata_sync_status.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream). Arguments are validated on the host before any
+ *     launch; an invalid call returns a status and launches nothing.
+ *   - Device pointers must be 16-byte aligned; d must be 16, 32 or 64.
+ *   - Errors: the return value is a kata_status. kata_last_error() gives a
+ *     one-line, thread-local description of the last failure on this thread.
+ *     Device-side failures (a bounded wait that ran out) set a per-device
+ *     error word that kata_sync_status() reads back and clears.
+ */
+#ifndef KATA_H
+#define KATA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define KATA_API __attribute__((visibility("default")))
+#else
+#define KATA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KATA_OK = 0,
+    KATA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+    KATA_ERR_UNSUPPORTED = 2, /* valid but not built: d, chunk or dtype */
+    KATA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    KATA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out */
+    KATA_ERR_WORKSPACE = 5    /* workspace missing or too small */
+} kata_status;
+
+typedef enum { KATA_F32 = 0, KATA_BF16 = 1 } kata_dtype; /* dtype of q, k, v */
+
+/* Library version (major*10000 + minor*100 + patch). */
+KATA_API int kata_version(void);
+/* Short name of a status code. */
+KATA_API const char *kata_status_string(int status);
+/* Description of the last failure on the calling thread ("" if none). */
+KATA_API const char *kata_last_error(void);
+/* D = d(d+1)/2. */
+KATA_API long kata_packed_dim(int d);
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads); a diagnostic for counting launches inside a timed region. */
+KATA_API unsigned long long kata_launch_count(void);
+
+/*
+ * Synchronise `stream`, then read and clear this device's error word.
+ * Returns KATA_OK, KATA_ERR_TIMEOUT (a kernel's bounded wait ran out and the
+ * kernel returned early: its outputs are invalid) or KATA_ERR_CUDA.
+ */
+KATA_API int kata_sync_status(void *stream);
+
+/* --------------------------------------------------------------- prefill -- */
+
+/* Device workspace bytes kata_prefill needs for these sizes (may be 0). */
+KATA_API size_t kata_prefill_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype);
+
+/*
+ * Causal chunked prefill [KATA s2.2, s2.3]:
+ *   o_i = phi(q_i)^T H_i / (phi(q_i)^T s_i + eps),
+ *   H_i = H_in + sum_{j<=i} phi(k_j) v_j^T,  s_i = s_in + sum_{j<=i} phi(k_j),
+ * computed chunk by chunk (chunk tokens at a time): inside a chunk the masked
+ * (Q K^T)^2 [V | 1] contraction, across chunks the carried state.
+ *
+ *   q, k, v   [B, H, T, d], dtype KATA_F32 or KATA_BF16.
+ *   H_in, s_in  initial state [B, H, D, d] / [B, H, D] fp32, packed layout;
+ *             both NULL = zero state; both or neither.
+ *   o         [B, H, T, d] fp32 output (NULL: state only).
+ *   H_out, s_out  final state, packed layout (NULL: not written; both or
+ *             neither). May alias H_in / s_in.
+ *   chunk     16, 32, 64 or 128; T must be a positive multiple of chunk.
+ *   workspace device scratch of at least kata_prefill_workspace_bytes().
+ * bf16 inputs run on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation and state); fp32 inputs run in fp32 on the CUDA cores.
+ */
+KATA_API int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
+                 int d, int chunk, float eps, const float *H_in, const float *s_in, float *o,
+                 float *H_out, float *s_out, void *workspace, size_t ws_bytes, void *stream);
+
+/* Which kernel kata_prefill runs for these sizes: 1 = tcgen05 tensor cores,
+ * 0 = CUDA cores, -1 = invalid or unsupported arguments. */
+KATA_API int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype);
+
+/* Device workspace for kata_prefill_host: staging for q, k, v and o plus
+ * kata_prefill_workspace_bytes(). */
+KATA_API size_t kata_prefill_host_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype);
+
+/*
+ * kata_prefill with host inputs and output: copies q_host, k_host, v_host to
+ * device staging inside `workspace`, runs kata_prefill on `stream` from a
+ * zero state, and copies o back to o_host (all asynchronous on `stream`;
+ * the caller synchronises before reading o_host).
+ */
+KATA_API int kata_prefill_host(const void *q_host, const void *k_host, const void *v_host, int dtype,
+                      int B, int H, int T, int d, int chunk, float eps, float *o_host,
+                      void *workspace, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- decode -- */
+
+/*
+ * One decode step per (b, h) [KATA s1 "constant-time recurrent inference"]:
+ *   H += phi(k) v^T;  s += phi(k);  o = phi(q)^T H / (phi(q)^T s + eps)
+ * (update first, then read out). The state is updated IN PLACE.
+ *   q, k, v   [B, H, d], dtype KATA_F32 or KATA_BF16.
+ *   Hst, s    [B, H, D, d] / [B, H, D] fp32, packed layout, read and written.
+ *   o         [B, H, d] fp32.
+ */
+KATA_API int kata_decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                     int d, float eps, float *Hst, float *s, float *o, void *stream);
+
+/*
+ * kata_decode_step with host q, k, v and o: staging (3 * B*H*d elements of
+ * dtype, then B*H*d fp32, each part 256-byte aligned) lives in `workspace`;
+ * the state stays on the device.
+ */
+KATA_API int kata_decode_step_host(const void *q_host, const void *k_host, const void *v_host,
+                          int dtype, int B, int H, int d, float eps, float *Hst, float *s,
+                          float *o_host, void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------ LoLA -- */
+
+/* Device workspace bytes lola_sre_score_topk needs. */
+KATA_API size_t lola_sre_workspace_bytes(int B, int H, int d, int n_cand);
+
+/*
+ * Self-recall error and top-k retention [LoLA "Self-Recall Error",
+ * "Inference strategy" steps 1-3]:
+ *   SRE_j = || phi(k_j)^T H / (phi(k_j)^T s + eps) - v_j ||^2
+ * for the n_cand candidates of every (b, h), scored against (Hst, s). The
+ * min(keep, n_cand) highest scores are kept (an exact tie goes to the smaller
+ * position); with merge = 1 every other candidate is added to the state,
+ * H += phi(k_j) v_j^T, s += phi(k_j).
+ *   Hst, s     [B, H, D, d] / [B, H, D] fp32 state to score against.
+ *   kc, vc     [B, H, n_cand, d] candidates, dtype KATA_F32 or KATA_BF16.
+ *   pos        [B, H, n_cand] int32 token positions, distinct within a head.
+ *   scores     [B, H, n_cand] fp32 SRE (NULL: not written).
+ *   keep_idx   [B, H, min(keep, n_cand)] int32 kept candidate slots in
+ *              ascending position.
+ *   Hst_mut, s_mut  merged state (merge = 1; may alias Hst / s; ignored when
+ *              merge = 0).
+ *   1 <= n_cand <= 1024, 0 <= keep.
+ */
+KATA_API int lola_sre_score_topk(const float *Hst, const float *s, const void *kc, const void *vc,
+                        const int *pos, int dtype, int B, int H, int d, int n_cand, int keep,
+                        float eps, int merge, float *scores, int *keep_idx, float *Hst_mut,
+                        float *s_mut, void *workspace, size_t ws_bytes, void *stream);
+
+/* Device workspace bytes lola_hybrid_readout needs. */
+KATA_API size_t lola_readout_workspace_bytes(int B, int H, int d, int nq);
+
+/*
+ * Hybrid readout of one segment [LoLA "Inference strategy" step 4,
+ * Methodology 1-3], one shared denominator:
+ *   o_i = [ sum_{j in W_i u S} exp(tau q_i.k_j) v_j + phi(q_i)^T H ]
+ *       / [ sum_{j in W_i u S} exp(tau q_i.k_j) + phi(q_i)^T s + eps ]
+ * for queries i = seg0 .. seg0+nq-1, window W_i = positions [w0, i] of k, v,
+ * sparse cache S = the first nc pairs of ck, cv.
+ *   q, k, v    [B, H, T, d] whole sequences, dtype KATA_F32 or KATA_BF16.
+ *   ck, cv     [B, H, cap, d] cache pairs, same dtype (nc <= cap).
+ *   Hst, s     state, packed layout.
+ *   o          [B, H, T, d] fp32; rows seg0 .. seg0+nq-1 are written.
+ *   0 <= w0 <= seg0, seg0 + nq <= T, 1 <= nq <= 256, seg0 + nq - w0 <= 1024.
+ */
+KATA_API int lola_hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                        int T, int d, int seg0, int nq, int w0, const void *ck,
+                        const void *cv, int nc, int cap, const float *Hst, const float *s,
+                        float eps, float tau, float *o, void *workspace, size_t ws_bytes,
+                        void *stream);
+
+/* Device workspace bytes lola_prefill needs. */
+KATA_API size_t lola_prefill_workspace_bytes(int B, int H, int T, int d, int window, int cache);
+
+/*
+ * The whole LoLA schedule over a sequence [LoLA "Inference strategy" 1-4],
+ * segment by segment (segment length = window):
+ *   for g = 0, 1, ...: read out segment g (lola_hybrid_readout with window
+ *   start max(0, window*(g-1))); then, for g >= 1, segment g-1 leaves the
+ *   window: its pairs and the cached pairs are scored by SRE against the
+ *   current state, the `cache` highest stay cached and the rest are merged.
+ *   q, k, v    [B, H, T, d]; T a positive multiple of window.
+ *   window     1..256; cache 0..1024 (window + cache <= 1024).
+ *   tau        softmax scale for window and cache pairs (1/sqrt(d) usual).
+ *   o          [B, H, T, d] fp32.
+ *   Hst, s     state in/out, packed layout (zero it for a fresh sequence).
+ *   kept_pos   optional [T/window - 1, B, H, cache] int32: the cached token
+ *              positions after each update, ascending, -1 padded (NULL: not
+ *              written).
+ */
+KATA_API int lola_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
+                 int d, int window, int cache, float eps, float tau, float *o, float *Hst,
+                 float *s, int *kept_pos, void *workspace, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KATA_H */

@@ -1,0 +1,28 @@
+"""Causal kernelized linear attention (rank-one PSD feature phi(x) = x x^T) and
+the LoLA self-recall-error sparse cache on NVIDIA B200 (sm_100a).
+
+The computation lives in libkata.so (C ABI: include/kata.h); this package is
+its thin Python binding plus the seeded synthetic input generators.
+"""
+from ._binding import (  # noqa: F401
+    KATA_BF16,
+    KATA_F32,
+    LIB_PATH,
+    SIGNATURES,
+    KataError,
+    decode_step,
+    decode_step_host,
+    hybrid_readout,
+    launch_count,
+    lib,
+    lola_prefill,
+    lola_prefill_workspace_bytes,
+    packed_dim,
+    prefill,
+    prefill_host,
+    prefill_host_workspace_bytes,
+    prefill_uses_tensor_cores,
+    prefill_workspace_bytes,
+    sre_score_topk,
+    sync_status,
+)

@@ -1,0 +1,405 @@
+// C ABI of libkata.so: argument validation, dispatch, status reporting.
+// The declarations and the contract of every entry point are in include/kata.h.
+#include <atomic>
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/kata.h"
+#include "kata_common.cuh"
+#include "kata_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int status, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(KATA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+__device__ unsigned int g_error_word;
+
+// Address of this device's error word (looked up once per device).
+unsigned int *error_word() {
+    static unsigned int *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned int *>(p);
+    }
+    return addr[dev];
+}
+
+std::atomic<unsigned long long> g_launches{0};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int dtype, int B, int H, int d) {
+    if (dtype != KATA_F32 && dtype != KATA_BF16)
+        return fail(KATA_ERR_UNSUPPORTED, "dtype %d is not KATA_F32 or KATA_BF16", dtype);
+    if (B <= 0 || H <= 0) return fail(KATA_ERR_INVALID_ARG, "B=%d H=%d must be positive", B, H);
+    if (d != 16 && d != 32 && d != 64)
+        return fail(KATA_ERR_UNSUPPORTED, "d=%d: only 16, 32 and 64 are built", d);
+    if ((long)B * H > (1L << 20)) return fail(KATA_ERR_INVALID_ARG, "B*H=%ld too large", (long)B * H);
+    return KATA_OK;
+}
+
+#define KATA_REQUIRE_PTR(p)                                                        \
+    do {                                                                           \
+        if (!(p)) return fail(KATA_ERR_INVALID_ARG, "%s must not be NULL", #p);    \
+        if (!aligned16(p))                                                         \
+            return fail(KATA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);    \
+    } while (0)
+
+#define KATA_OPTIONAL_PTR(p)                                                       \
+    do {                                                                           \
+        if ((p) && !aligned16(p))                                                  \
+            return fail(KATA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);    \
+    } while (0)
+
+size_t elem_bytes(int dtype) { return dtype == KATA_F32 ? 4 : 2; }
+
+}  // namespace
+
+cudaError_t kata::after_launch() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
+extern "C" {
+
+unsigned long long kata_launch_count(void) { return g_launches.load(); }
+
+int kata_version(void) { return 100; }
+
+const char *kata_status_string(int status) {
+    switch (status) {
+        case KATA_OK: return "KATA_OK";
+        case KATA_ERR_INVALID_ARG: return "KATA_ERR_INVALID_ARG";
+        case KATA_ERR_UNSUPPORTED: return "KATA_ERR_UNSUPPORTED";
+        case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
+        case KATA_ERR_TIMEOUT: return "KATA_ERR_TIMEOUT";
+        case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
+        default: return "KATA_ERR_UNKNOWN";
+    }
+}
+
+const char *kata_last_error(void) { return g_last_error; }
+
+long kata_packed_dim(int d) { return (long)d * (d + 1) / 2; }
+
+int kata_sync_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int *w = error_word();
+    if (!w) return fail(KATA_ERR_CUDA, "error word unavailable");
+    unsigned int h = 0;
+    e = cudaMemcpy(&h, w, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "read error word");
+    if (h != kata::kErrNone) {
+        unsigned int zero = 0;
+        e = cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+        return fail(KATA_ERR_TIMEOUT, "a kernel's bounded wait ran out (code %u)", h);
+    }
+    return KATA_OK;
+}
+
+/* ------------------------------------------------------------- prefill --- */
+
+static int check_prefill(int dtype, int B, int H, int T, int d, int chunk) {
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128)
+        return fail(KATA_ERR_UNSUPPORTED, "chunk=%d: only 16, 32, 64, 128", chunk);
+    if (T <= 0 || T % chunk)
+        return fail(KATA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk=%d", T, chunk);
+    if ((long)T > (1L << 24)) return fail(KATA_ERR_INVALID_ARG, "T=%d too large", T);
+    return KATA_OK;
+}
+
+static size_t prefill_ws_bytes(int B, int H, int T, int d, int chunk, int dtype) {
+    // a copy of s_in, used when s_out aliases it
+    size_t b = kata::align_up((size_t)B * H * kata::packed_dim(d) * sizeof(float), 256);
+    if (dtype == KATA_BF16) b += kata::prefill_tc_workspace_bytes(B, H, T, d, chunk);
+    return b;
+}
+
+size_t kata_prefill_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype) {
+    if (check_prefill(dtype, B, H, T, d, chunk)) return 0;
+    return prefill_ws_bytes(B, H, T, d, chunk, dtype);
+}
+
+int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
+                 int d, int chunk, float eps, const float *H_in, const float *s_in, float *o,
+                 float *H_out, float *s_out, void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_prefill(dtype, B, H, T, d, chunk);
+    if (st) return st;
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_OPTIONAL_PTR(o);
+    KATA_OPTIONAL_PTR(H_in);
+    KATA_OPTIONAL_PTR(s_in);
+    KATA_OPTIONAL_PTR(H_out);
+    KATA_OPTIONAL_PTR(s_out);
+    if (!H_in != !s_in) return fail(KATA_ERR_INVALID_ARG, "H_in and s_in: both or neither");
+    if (!H_out != !s_out) return fail(KATA_ERR_INVALID_ARG, "H_out and s_out: both or neither");
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = prefill_ws_bytes(B, H, T, d, chunk, dtype);
+    if (ws_bytes < need || (need && !workspace))
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_OPTIONAL_PTR(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int *err = error_word();
+    if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
+
+    const size_t s_bytes = (size_t)B * H * kata::packed_dim(d) * sizeof(float);
+    char *ws = static_cast<char *>(workspace);
+    if (s_in && s_out == s_in) {  // every CTA of a head reads s_in: keep a copy
+        cudaError_t e = cudaMemcpyAsync(ws, s_in, s_bytes, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "copy s_in");
+        s_in = reinterpret_cast<const float *>(ws);
+    }
+    kata::PrefillArgs a{q, k, v, dtype, B, H, T, d, chunk, eps, H_in, s_in, o, H_out, s_out,
+                        ws + kata::align_up(s_bytes, 256), ws_bytes - kata::align_up(s_bytes, 256),
+                        err};
+    cudaError_t e;
+    if (dtype == KATA_BF16 && kata::prefill_tc_supported(a))
+        e = kata::prefill_tc(a, s);
+    else
+        e = kata::prefill_simt(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_prefill launch");
+    return KATA_OK;
+}
+
+int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype) {
+    if (check_prefill(dtype, B, H, T, d, chunk)) return -1;
+    kata::PrefillArgs a{};
+    a.dtype = dtype;
+    a.B = B;
+    a.H = H;
+    a.T = T;
+    a.d = d;
+    a.chunk = chunk;
+    return dtype == KATA_BF16 && kata::prefill_tc_supported(a) ? 1 : 0;
+}
+
+size_t kata_prefill_host_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype) {
+    if (check_prefill(dtype, B, H, T, d, chunk)) return 0;
+    const size_t n = (size_t)B * H * T * d;
+    return 3 * kata::align_up(n * elem_bytes(dtype), 256) + kata::align_up(n * 4, 256) +
+           prefill_ws_bytes(B, H, T, d, chunk, dtype);
+}
+
+int kata_prefill_host(const void *q_host, const void *k_host, const void *v_host, int dtype,
+                      int B, int H, int T, int d, int chunk, float eps, float *o_host,
+                      void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_prefill(dtype, B, H, T, d, chunk);
+    if (st) return st;
+    if (!q_host || !k_host || !v_host || !o_host)
+        return fail(KATA_ERR_INVALID_ARG, "host pointers must not be NULL");
+    const size_t need = kata_prefill_host_workspace_bytes(B, H, T, d, chunk, dtype);
+    if (!workspace || ws_bytes < need)
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_REQUIRE_PTR(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)B * H * T * d, xb = n * elem_bytes(dtype);
+    char *w = static_cast<char *>(workspace);
+    char *qd = w, *kd = qd + kata::align_up(xb, 256), *vd = kd + kata::align_up(xb, 256);
+    float *od = reinterpret_cast<float *>(vd + kata::align_up(xb, 256));
+    char *rest = reinterpret_cast<char *>(od) + kata::align_up(n * 4, 256);
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(qd, q_host, xb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(kd, k_host, xb, cudaMemcpyHostToDevice, s)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(vd, v_host, xb, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        return cuda_fail(e, "host-to-device copy");
+    st = kata_prefill(qd, kd, vd, dtype, B, H, T, d, chunk, eps, nullptr, nullptr, od, nullptr,
+                      nullptr, rest, ws_bytes - (size_t)(rest - w), stream);
+    if (st) return st;
+    if ((e = cudaMemcpyAsync(o_host, od, n * 4, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+        return cuda_fail(e, "device-to-host copy");
+    return KATA_OK;
+}
+
+/* -------------------------------------------------------------- decode --- */
+
+int kata_decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                     int d, float eps, float *Hst, float *s, float *o, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_REQUIRE_PTR(o);
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    cudaError_t e = kata::decode_step(q, k, v, dtype, B, H, d, eps, Hst, s, o,
+                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kata_decode_step launch");
+    return KATA_OK;
+}
+
+int kata_decode_step_host(const void *q_host, const void *k_host, const void *v_host,
+                          int dtype, int B, int H, int d, float eps, float *Hst, float *s,
+                          float *o_host, void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (!q_host || !k_host || !v_host || !o_host)
+        return fail(KATA_ERR_INVALID_ARG, "host pointers must not be NULL");
+    const size_t n = (size_t)B * H * d, xb = n * elem_bytes(dtype);
+    const size_t need = 3 * kata::align_up(xb, 256) + kata::align_up(n * 4, 256);
+    if (!workspace || ws_bytes < need)
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_REQUIRE_PTR(workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    char *qd = static_cast<char *>(workspace), *kd = qd + kata::align_up(xb, 256);
+    char *vd = kd + kata::align_up(xb, 256);
+    float *od = reinterpret_cast<float *>(vd + kata::align_up(xb, 256));
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(qd, q_host, xb, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(kd, k_host, xb, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(vd, v_host, xb, cudaMemcpyHostToDevice, cs)) != cudaSuccess)
+        return cuda_fail(e, "host-to-device copy");
+    st = kata_decode_step(qd, kd, vd, dtype, B, H, d, eps, Hst, s, od, stream);
+    if (st) return st;
+    if ((e = cudaMemcpyAsync(o_host, od, n * 4, cudaMemcpyDeviceToHost, cs)) != cudaSuccess)
+        return cuda_fail(e, "device-to-host copy");
+    return KATA_OK;
+}
+
+/* ---------------------------------------------------------------- LoLA --- */
+
+size_t lola_sre_workspace_bytes(int B, int H, int d, int n_cand) {
+    if (check_common(KATA_F32, B, H, d) || n_cand < 1 || n_cand > 1024) return 0;
+    return kata::sre_workspace_bytes(B, H, d, n_cand);
+}
+
+int lola_sre_score_topk(const float *Hst, const float *s, const void *kc, const void *vc,
+                        const int *pos, int dtype, int B, int H, int d, int n_cand, int keep,
+                        float eps, int merge, float *scores, int *keep_idx, float *Hst_mut,
+                        float *s_mut, void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (n_cand < 1 || n_cand > 1024)
+        return fail(KATA_ERR_INVALID_ARG, "n_cand=%d must be in [1, 1024]", n_cand);
+    if (keep < 0) return fail(KATA_ERR_INVALID_ARG, "keep=%d must be >= 0", keep);
+    if (merge != 0 && merge != 1) return fail(KATA_ERR_INVALID_ARG, "merge must be 0 or 1");
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_REQUIRE_PTR(kc);
+    KATA_REQUIRE_PTR(vc);
+    KATA_REQUIRE_PTR(pos);
+    KATA_OPTIONAL_PTR(scores);
+    if (keep > 0) KATA_REQUIRE_PTR(keep_idx);
+    if (merge) {
+        KATA_REQUIRE_PTR(Hst_mut);
+        KATA_REQUIRE_PTR(s_mut);
+    }
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = kata::sre_workspace_bytes(B, H, d, n_cand);
+    if (!workspace || ws_bytes < need)
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_REQUIRE_PTR(workspace);
+    cudaError_t e = kata::sre_score_topk(Hst, s, kc, vc, pos, dtype, B, H, d, n_cand, n_cand,
+                                         keep, eps, merge, scores, keep_idx, Hst_mut, s_mut,
+                                         workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "lola_sre_score_topk launch");
+    return KATA_OK;
+}
+
+size_t lola_readout_workspace_bytes(int B, int H, int d, int nq) {
+    if (check_common(KATA_F32, B, H, d) || nq < 1 || nq > 256) return 0;
+    return kata::readout_workspace_bytes(B, H, d, nq);
+}
+
+int lola_hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                        int T, int d, int seg0, int nq, int w0, const void *ck,
+                        const void *cv, int nc, int cap, const float *Hst, const float *s,
+                        float eps, float tau, float *o, void *workspace, size_t ws_bytes,
+                        void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (T <= 0 || nq < 1 || nq > 256 || seg0 < 0 || seg0 + nq > T || w0 < 0 || w0 > seg0 ||
+        seg0 + nq - w0 > 1024)
+        return fail(KATA_ERR_INVALID_ARG, "bad segment T=%d seg0=%d nq=%d w0=%d", T, seg0, nq, w0);
+    if (nc < 0 || cap < nc || cap > 4096)
+        return fail(KATA_ERR_INVALID_ARG, "bad cache nc=%d cap=%d", nc, cap);
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_REQUIRE_PTR(o);
+    if (nc > 0) {
+        KATA_REQUIRE_PTR(ck);
+        KATA_REQUIRE_PTR(cv);
+    }
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = kata::readout_workspace_bytes(B, H, d, nq);
+    if (!workspace || ws_bytes < need)
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_REQUIRE_PTR(workspace);
+    cudaError_t e = kata::hybrid_readout(q, k, v, dtype, B, H, T, d, seg0, nq, w0, ck, cv, nc,
+                                         cap, Hst, s, eps, tau, o, workspace, ws_bytes,
+                                         static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "lola_hybrid_readout launch");
+    return KATA_OK;
+}
+
+size_t lola_prefill_workspace_bytes(int B, int H, int T, int d, int window, int cache) {
+    if (check_common(KATA_F32, B, H, d) || window < 1 || window > 256 || cache < 0 ||
+        window + cache > 1024)
+        return 0;
+    return kata::lola_workspace_bytes(B, H, T, d, window, cache);
+}
+
+int lola_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
+                 int d, int window, int cache, float eps, float tau, float *o, float *Hst,
+                 float *s, int *kept_pos, void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (window < 1 || window > 256 || cache < 0 || window + cache > 1024)
+        return fail(KATA_ERR_INVALID_ARG, "window=%d cache=%d out of range", window, cache);
+    if (T <= 0 || T % window)
+        return fail(KATA_ERR_INVALID_ARG, "T=%d must be a positive multiple of window=%d", T, window);
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_REQUIRE_PTR(o);
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_OPTIONAL_PTR(kept_pos);
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = kata::lola_workspace_bytes(B, H, T, d, window, cache);
+    if (!workspace || ws_bytes < need)
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    KATA_REQUIRE_PTR(workspace);
+    cudaError_t e = kata::lola_run(q, k, v, dtype, B, H, T, d, window, cache, eps, tau, o, Hst,
+                                   s, kept_pos, workspace, ws_bytes,
+                                   static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "lola_prefill launch");
+    return KATA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Host-side interfaces between the C ABI (kata_abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kata {
+
+struct PrefillArgs {
+    const void *q, *k, *v;
+    int dtype;  // 0 = fp32, 1 = bf16
+    int B, H, T, d, chunk;
+    float eps;
+    const float *H_in, *s_in;
+    float *o, *H_out, *s_out;
+    void *ws;
+    size_t ws_bytes;
+    unsigned int *err;  // per-device error word
+};
+
+// fp32 CUDA-core path: any supported d and chunk, fp32 or bf16 inputs.
+cudaError_t prefill_simt(const PrefillArgs &a, cudaStream_t stream);
+
+// tcgen05 tensor-core path (bf16 inputs). Returns cudaErrorNotSupported when
+// the shape is not one it takes; the caller then uses the CUDA-core path.
+bool prefill_tc_supported(const PrefillArgs &a);
+size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
+cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream);
+
+cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                        int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream);
+
+// LoLA pieces (lola.cu).
+size_t sre_workspace_bytes(int B, int H, int d, int n_cand);
+cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, const void *vc,
+                           const int *pos, int dtype, int B, int H, int d, int n_cand,
+                           int cand_stride, int keep, float eps, int merge, float *scores,
+                           int *keep_idx, float *Hst_mut, float *s_mut, void *ws,
+                           size_t ws_bytes, cudaStream_t stream);
+size_t readout_workspace_bytes(int B, int H, int d, int nq);
+cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B,
+                           int H, int T, int d, int seg0, int nq, int w0, const void *ck,
+                           const void *cv, int nc, int cap, const float *Hst, const float *s,
+                           float eps, float tau, float *o, void *ws, size_t ws_bytes,
+                           cudaStream_t stream);
+size_t lola_workspace_bytes(int B, int H, int T, int d, int window, int cache);
+cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                     int T, int d, int window, int cache, float eps, float tau, float *o,
+                     float *Hst, float *s, int *kept_pos, void *ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Called right after every kernel launch: counts it (kata_launch_count) and
+// returns the launch status.
+cudaError_t after_launch();
+
+}  // namespace kata

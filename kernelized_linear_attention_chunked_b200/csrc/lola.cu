@@ -1,0 +1,591 @@
+// LoLA sparse-cache pieces on the CUDA cores, fp32 arithmetic.
+//
+// "LoLA: Low-Rank Linear Attention with Sparse Caching":
+//  - "Self-Recall Error": SRE(k, v | H, s) = || phi(k)^T H / phi(k)^T s - v ||^2
+//    (eps added to the denominator, as in every readout here);
+//  - "Inference strategy" 1-3: score the pairs leaving the window together
+//    with the cached pairs, keep the highest SRE in the cache, merge the rest
+//    into the linear state by outer-product updates;
+//  - "Inference strategy" 4 / Methodology 1-3: the output combines window
+//    softmax attention, sparse-cache attention and the linear-state readout.
+// phi is the rank-one PSD feature of "Kernelized Linear Attention: Breaking
+// the Capacity Wall with Symmetric Cones", s2.2.
+//
+// Kernels:
+//  state_partial  phi(x_i)^T [H | s] for many rows x_i, split over slices of
+//                 the packed dimension (one CTA per head x slice x 64 rows);
+//                 partial sums go to the workspace and are reduced in a fixed
+//                 order by the consumer, so results are run-to-run identical.
+//  sre_select     reduce partials, SRE per candidate, rank-based top-k (every
+//                 thread counts the candidates ranked before it), kept slots
+//                 in ascending position, list of slots to merge.
+//  merge          H_dst = H_src + sum_{j merged} phi(k_j) v_j^T per slice.
+//  hybrid_finish  window + cache softmax terms, plus the state partials, one
+//                 shared denominator.
+//  append/compact the cache bookkeeping of the schedule.
+#include "kata_common.cuh"
+#include "kata_internal.h"
+
+namespace kata {
+namespace {
+
+constexpr int kRows = 64;
+constexpr int kThreads = 256;
+constexpr int kMaxSlice = 512;
+constexpr int kTargetCtas = 296;  // two CTAs per SM on a 148-SM part
+
+int num_slices(int nh, int n, int d) {
+    const int D = packed_dim(d);
+    const int rb = (n + kRows - 1) / kRows;
+    const int pmin = (D + kMaxSlice - 1) / kMaxSlice;
+    const int pmax = (D + 63) / 64;
+    int p = (kTargetCtas + nh * rb - 1) / (nh * rb);
+    if (p < pmin) p = pmin;
+    if (p > pmax) p = pmax;
+    return p;
+}
+
+size_t partial_floats(int nh, int n, int d) {
+    return (size_t)num_slices(nh, n, d) * nh * n * (d + 1);
+}
+
+size_t state_partial_smem(int d, int P) {
+    const int D = packed_dim(d);
+    const int slice = (D + P - 1) / P;
+    return ((size_t)kRows * (d + 1) + (size_t)slice * d + slice) * sizeof(float) +
+           align_up((size_t)D * sizeof(uint16_t), 16);
+}
+
+// part[p][h][i][e] = sum_{r in slice p} phi(x_i)_r H[r][e]; part[..][d] uses s.
+template <typename Tin, int DH>
+__global__ void __launch_bounds__(kThreads)
+state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
+                     const float *__restrict__ Hst, const float *__restrict__ s, int P,
+                     float *__restrict__ part) {
+    constexpr int D = DH * (DH + 1) / 2;
+    constexpr int EQ = DH / 4;
+    const int h = blockIdx.x, p = blockIdx.y, i0 = blockIdx.z * kRows;
+    const int nh = gridDim.x;
+    const int slice = (D + P - 1) / P;
+    const int r0 = p * slice, r1 = min(D, r0 + slice), nr = max(0, r1 - r0);
+    const int tid = threadIdx.x;
+
+    extern __shared__ float4 smem4[];
+    float *Xs = reinterpret_cast<float *>(smem4);  // [kRows][DH+1]
+    float *Hsl = Xs + kRows * (DH + 1);            // [slice][DH]
+    float *ssl = Hsl + (size_t)slice * DH;         // [slice]
+    uint16_t *tab = reinterpret_cast<uint16_t *>(ssl + slice);
+
+    build_pair_table(tab, DH);
+    const Tin *Xh = X + (size_t)h * x_head_stride;
+    for (int idx = tid; idx < kRows * DH; idx += kThreads) {
+        const int i = idx / DH, a = idx % DH;
+        Xs[i * (DH + 1) + a] = (i0 + i < n) ? to_f32(Xh[(size_t)(i0 + i) * DH + a]) : 0.f;
+    }
+    const float4 *H4 = reinterpret_cast<const float4 *>(Hst + ((size_t)h * D + r0) * DH);
+    float4 *Hs4 = reinterpret_cast<float4 *>(Hsl);
+    for (int idx = tid; idx < nr * DH / 4; idx += kThreads) Hs4[idx] = H4[idx];
+    for (int idx = tid; idx < nr; idx += kThreads) ssl[idx] = s[(size_t)h * D + r0 + idx];
+    __syncthreads();
+
+    const int i = tid >> 2, eq = (tid & 3) * EQ;
+    const float *xi = Xs + i * (DH + 1);
+    float acc[EQ];
+#pragma unroll
+    for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
+    float den = 0.f;
+    for (int rr = 0; rr < nr; ++rr) {
+        const float ph = phi_entry(xi, tab[r0 + rr]);
+        const float4 *hr = reinterpret_cast<const float4 *>(Hsl + (size_t)rr * DH + eq);
+#pragma unroll
+        for (int c = 0; c < EQ / 4; ++c) {
+            const float4 hv = hr[c];
+            acc[4 * c + 0] = fmaf(ph, hv.x, acc[4 * c + 0]);
+            acc[4 * c + 1] = fmaf(ph, hv.y, acc[4 * c + 1]);
+            acc[4 * c + 2] = fmaf(ph, hv.z, acc[4 * c + 2]);
+            acc[4 * c + 3] = fmaf(ph, hv.w, acc[4 * c + 3]);
+        }
+        den = fmaf(ph, ssl[rr], den);
+    }
+    if (i0 + i < n) {
+        float *dst = part + (((size_t)p * nh + h) * n + i0 + i) * (DH + 1);
+#pragma unroll
+        for (int c = 0; c < EQ; ++c) dst[eq + c] = acc[c];
+        if (eq == 0) dst[DH] = den;
+    }
+}
+
+template <typename Tin>
+cudaError_t launch_state_partial(const Tin *X, long x_head_stride, int nh, int n, int d,
+                                 const float *Hst, const float *s, int P, float *part,
+                                 cudaStream_t stream) {
+    const size_t smem = state_partial_smem(d, P);
+    dim3 grid(nh, P, (n + kRows - 1) / kRows);
+    cudaError_t err;
+#define KATA_LAUNCH_PARTIAL(DH)                                                               \
+    err = cudaFuncSetAttribute(state_partial_kernel<Tin, DH>,                                 \
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
+    if (err != cudaSuccess) return err;                                                       \
+    state_partial_kernel<Tin, DH><<<grid, kThreads, smem, stream>>>(X, x_head_stride, n, Hst, \
+                                                                     s, P, part);
+    switch (d) {
+        case 16: KATA_LAUNCH_PARTIAL(16) break;
+        case 32: KATA_LAUNCH_PARTIAL(32) break;
+        case 64: KATA_LAUNCH_PARTIAL(64) break;
+        default: return cudaErrorInvalidValue;
+    }
+#undef KATA_LAUNCH_PARTIAL
+    return after_launch();
+}
+
+// Candidate i is retained before candidate j: higher SRE, then smaller
+// position, then smaller slot.
+__device__ __forceinline__ bool retained_before(float si, int pi, int i, float sj, int pj,
+                                                int j) {
+    if (si != sj) return si > sj;
+    if (pi != pj) return pi < pj;
+    return i < j;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(1024)
+sre_select_kernel(const float *__restrict__ part, int P, int n, int d,
+                  const Tin *__restrict__ vc, long cand_head_stride,
+                  const int *__restrict__ pos, long pos_head_stride, int keep, float eps,
+                  float *__restrict__ scores, int *__restrict__ keep_idx,
+                  int *__restrict__ mlist, int *__restrict__ mcount) {
+    __shared__ float sc[1024];
+    __shared__ int ps[1024];
+    __shared__ unsigned char kept[1024];
+    const int h = blockIdx.x, nh = gridDim.x, j = threadIdx.x;
+    const int m = keep < n ? keep : n;
+    if (j < n) {
+        float den = 0.f;
+        for (int p = 0; p < P; ++p) den += part[(((size_t)p * nh + h) * n + j) * (d + 1) + d];
+        const float inv = 1.f / (den + eps);
+        const Tin *vj = vc + (size_t)h * cand_head_stride + (size_t)j * d;
+        float err = 0.f;
+        for (int e = 0; e < d; ++e) {
+            float num = 0.f;
+            for (int p = 0; p < P; ++p) num += part[(((size_t)p * nh + h) * n + j) * (d + 1) + e];
+            const float diff = num * inv - to_f32(vj[e]);
+            err = fmaf(diff, diff, err);
+        }
+        sc[j] = isnan(err) ? -INFINITY : err;  // a total order even for 0/0 scores
+        ps[j] = pos[(size_t)h * pos_head_stride + j];
+    }
+    __syncthreads();
+    bool isk = false;
+    if (j < n) {
+        int rank = 0;
+        for (int i = 0; i < n; ++i) rank += retained_before(sc[i], ps[i], i, sc[j], ps[j], j);
+        isk = rank < m;
+        kept[j] = isk;
+    }
+    __syncthreads();
+    if (j < n) {
+        if (isk) {
+            int pr = 0;
+            for (int i = 0; i < n; ++i)
+                pr += kept[i] && (ps[i] < ps[j] || (ps[i] == ps[j] && i < j));
+            if (pr < m) keep_idx[(size_t)h * m + pr] = j;
+        } else {
+            int mr = 0;
+            for (int i = 0; i < j; ++i) mr += !kept[i];
+            if (mr < n - m) mlist[(size_t)h * n + mr] = j;
+        }
+        if (scores) scores[(size_t)h * n + j] = sc[j];
+    }
+    if (j == 0) mcount[h] = n - m;
+}
+
+template <typename Tin, int DH>
+__global__ void __launch_bounds__(kThreads)
+merge_kernel(const float *Hsrc, const float *ssrc, float *Hdst, float *sdst,
+             const Tin *__restrict__ kc, const Tin *__restrict__ vc, long cand_head_stride,
+             const int *__restrict__ mlist, const int *__restrict__ mcount, int n, int P) {
+    constexpr int D = DH * (DH + 1) / 2;
+    constexpr int EQ = DH / 4;
+    __shared__ float Ks[kRows][DH + 1];
+    __shared__ float Vs[kRows][DH];
+    __shared__ uint16_t tab[D];
+    const int h = blockIdx.x, p = blockIdx.y, tid = threadIdx.x;
+    const int slice = (D + P - 1) / P;
+    const int r0 = p * slice, r1 = min(D, r0 + slice);
+    const int m = mcount[h];
+    build_pair_table(tab, DH);
+    const Tin *kh = kc + (size_t)h * cand_head_stride;
+    const Tin *vh = vc + (size_t)h * cand_head_stride;
+    const int eq = (tid & 3) * EQ;
+    for (int rb = r0; rb < r1; rb += kRows) {
+        const int r = rb + (tid >> 2);
+        float acc[EQ];
+#pragma unroll
+        for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
+        float sacc = 0.f;
+        for (int mb = 0; mb < m; mb += kRows) {
+            const int nb = min(kRows, m - mb);
+            __syncthreads();
+            for (int idx = tid; idx < nb * DH; idx += kThreads) {
+                const int ii = idx / DH, a = idx % DH;
+                const int j = mlist[(size_t)h * n + mb + ii];
+                Ks[ii][a] = to_f32(kh[(size_t)j * DH + a]);
+                Vs[ii][a] = to_f32(vh[(size_t)j * DH + a]);
+            }
+            __syncthreads();
+            if (r < r1) {
+                const uint16_t ab = tab[r];
+                for (int ii = 0; ii < nb; ++ii) {
+                    const float pk = phi_entry(Ks[ii], ab);
+                    sacc += pk;
+#pragma unroll
+                    for (int c = 0; c < EQ; ++c) acc[c] = fmaf(pk, Vs[ii][eq + c], acc[c]);
+                }
+            }
+        }
+        if (r < r1) {
+            const size_t base = ((size_t)h * D + r) * DH + eq;
+#pragma unroll
+            for (int c = 0; c < EQ; ++c) Hdst[base + c] = Hsrc[base + c] + acc[c];
+            if (eq == 0) sdst[(size_t)h * D + r] = ssrc[(size_t)h * D + r] + sacc;
+        }
+    }
+}
+
+// One warp per query: window and cache softmax terms plus the state partials.
+template <typename Tin, int DH>
+__global__ void __launch_bounds__(kThreads)
+hybrid_finish_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                     const Tin *__restrict__ v, int T, int seg0, int nq, int w0,
+                     const Tin *__restrict__ ck, const Tin *__restrict__ cv, int nc, int cap,
+                     const float *__restrict__ part, int P, float eps, float tau,
+                     float *__restrict__ o) {
+    constexpr int PL = (DH + 31) / 32;  // elements per lane
+    const int h = blockIdx.x, nh = gridDim.x;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int r = blockIdx.y * (kThreads / 32) + warp;
+    if (r >= nq) return;
+    const int i = seg0 + r;
+    const size_t hoff = (size_t)h * T * DH;
+    float qv[PL], num[PL];
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        const int a = lane + 32 * c;
+        qv[c] = a < DH ? to_f32(q[hoff + (size_t)i * DH + a]) : 0.f;
+        num[c] = 0.f;
+    }
+    float den = 0.f;
+    const int nw = i - w0 + 1;
+    for (int jj = 0; jj < nw + nc; ++jj) {
+        const Tin *kj, *vj;
+        if (jj < nw) {
+            kj = k + hoff + (size_t)(w0 + jj) * DH;
+            vj = v + hoff + (size_t)(w0 + jj) * DH;
+        } else {
+            kj = ck + ((size_t)h * cap + (jj - nw)) * DH;
+            vj = cv + ((size_t)h * cap + (jj - nw)) * DH;
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            const int a = lane + 32 * c;
+            if (a < DH) dot = fmaf(qv[c], to_f32(kj[a]), dot);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        const float w = expf(tau * dot);
+        den += w;
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            const int a = lane + 32 * c;
+            if (a < DH) num[c] = fmaf(w, to_f32(vj[a]), num[c]);
+        }
+    }
+    for (int p = 0; p < P; ++p) {
+        const float *src = part + (((size_t)p * nh + h) * nq + r) * (DH + 1);
+        den += src[DH];
+#pragma unroll
+        for (int c = 0; c < PL; ++c) {
+            const int a = lane + 32 * c;
+            if (a < DH) num[c] += src[a];
+        }
+    }
+    const float inv = 1.f / (den + eps);
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {
+        const int a = lane + 32 * c;
+        if (a < DH) o[hoff + (size_t)i * DH + a] = num[c] * inv;
+    }
+}
+
+template <typename Tin>
+__global__ void lola_append_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, int T,
+                                   int d, int pstart, int U, Tin *cand_k, Tin *cand_v,
+                                   int *cand_pos, int cap, int nc) {
+    const int h = blockIdx.x;
+    for (int idx = threadIdx.x; idx < U * d; idx += blockDim.x) {
+        const int u = idx / d, a = idx % d;
+        const size_t src = ((size_t)h * T + pstart + u) * d + a;
+        const size_t dst = ((size_t)h * cap + nc + u) * d + a;
+        cand_k[dst] = k[src];
+        cand_v[dst] = v[src];
+        if (a == 0) cand_pos[(size_t)h * cap + nc + u] = pstart + u;
+    }
+}
+
+template <typename Tin>
+__global__ void lola_compact_kernel(const Tin *__restrict__ src_k, const Tin *__restrict__ src_v,
+                                    const int *__restrict__ src_pos, Tin *__restrict__ dst_k,
+                                    Tin *__restrict__ dst_v, int *__restrict__ dst_pos,
+                                    const int *__restrict__ keep_idx, int m, int cap, int d,
+                                    int *__restrict__ kept_pos, int cache) {
+    const int h = blockIdx.x;
+    for (int idx = threadIdx.x; idx < m * d; idx += blockDim.x) {
+        const int rr = idx / d, a = idx % d;
+        const int j = keep_idx[(size_t)h * m + rr];
+        dst_k[((size_t)h * cap + rr) * d + a] = src_k[((size_t)h * cap + j) * d + a];
+        dst_v[((size_t)h * cap + rr) * d + a] = src_v[((size_t)h * cap + j) * d + a];
+        if (a == 0) dst_pos[(size_t)h * cap + rr] = src_pos[(size_t)h * cap + j];
+    }
+    if (kept_pos)
+        for (int rr = threadIdx.x; rr < cache; rr += blockDim.x)
+            kept_pos[(size_t)h * cache + rr] =
+                rr < m ? src_pos[(size_t)h * cap + keep_idx[(size_t)h * m + rr]] : -1;
+}
+
+size_t elem_size(int dtype) { return dtype == 0 ? 4 : 2; }
+
+struct SreWs {
+    float *part;
+    int *mlist, *mcount;
+};
+
+SreWs carve_sre(void *ws, int nh, int n, int d) {
+    char *p = static_cast<char *>(ws);
+    SreWs w;
+    w.part = reinterpret_cast<float *>(p);
+    p += align_up(partial_floats(nh, n, d) * sizeof(float), 256);
+    w.mlist = reinterpret_cast<int *>(p);
+    p += align_up((size_t)nh * n * sizeof(int), 256);
+    w.mcount = reinterpret_cast<int *>(p);
+    return w;
+}
+
+template <typename Tin>
+cudaError_t sre_impl(const float *Hst, const float *s, const Tin *kc, const Tin *vc,
+                     const int *pos, int nh, int d, int n, int cand_stride, int keep, float eps,
+                     int merge, float *scores, int *keep_idx, float *Hst_mut, float *s_mut,
+                     void *ws, cudaStream_t stream) {
+    const int P = num_slices(nh, n, d);
+    SreWs w = carve_sre(ws, nh, n, d);
+    const long cstride = (long)cand_stride * d;
+    cudaError_t err = launch_state_partial<Tin>(kc, cstride, nh, n, d, Hst, s, P, w.part, stream);
+    if (err != cudaSuccess) return err;
+    const int threads = ((n + 31) / 32) * 32;
+    sre_select_kernel<Tin><<<nh, threads, 0, stream>>>(w.part, P, n, d, vc, cstride, pos,
+                                                       cand_stride, keep, eps, scores, keep_idx,
+                                                       w.mlist, w.mcount);
+    if ((err = after_launch()) != cudaSuccess) return err;
+    if (!merge || keep >= n) {
+        if (merge && (Hst_mut != Hst || s_mut != s)) {  // nothing to merge: copy through
+            const int D = packed_dim(d);
+            if ((err = cudaMemcpyAsync(Hst_mut, Hst, (size_t)nh * D * d * 4,
+                                       cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
+                return err;
+            if ((err = cudaMemcpyAsync(s_mut, s, (size_t)nh * D * 4, cudaMemcpyDeviceToDevice,
+                                       stream)) != cudaSuccess)
+                return err;
+        }
+        return cudaSuccess;
+    }
+    const int D = packed_dim(d);
+    const int P2 = (D + 127) / 128;
+    dim3 grid(nh, P2);
+    switch (d) {
+        case 16: merge_kernel<Tin, 16><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
+        case 32: merge_kernel<Tin, 32><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
+        case 64: merge_kernel<Tin, 64><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return after_launch();
+}
+
+template <typename Tin>
+cudaError_t readout_impl(const Tin *q, const Tin *k, const Tin *v, int nh, int T, int d,
+                         int seg0, int nq, int w0, const Tin *ck, const Tin *cv, int nc,
+                         int cap, const float *Hst, const float *s, float eps, float tau,
+                         float *o, void *ws, cudaStream_t stream) {
+    const int P = num_slices(nh, nq, d);
+    float *part = static_cast<float *>(ws);
+    cudaError_t err = launch_state_partial<Tin>(q + (size_t)seg0 * d, (long)T * d, nh, nq, d,
+                                                Hst, s, P, part, stream);
+    if (err != cudaSuccess) return err;
+    dim3 grid(nh, (nq + 7) / 8);
+    switch (d) {
+        case 16: hybrid_finish_kernel<Tin, 16><<<grid, kThreads, 0, stream>>>(q, k, v, T, seg0, nq, w0, ck, cv, nc, cap, part, P, eps, tau, o); break;
+        case 32: hybrid_finish_kernel<Tin, 32><<<grid, kThreads, 0, stream>>>(q, k, v, T, seg0, nq, w0, ck, cv, nc, cap, part, P, eps, tau, o); break;
+        case 64: hybrid_finish_kernel<Tin, 64><<<grid, kThreads, 0, stream>>>(q, k, v, T, seg0, nq, w0, ck, cv, nc, cap, part, P, eps, tau, o); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return after_launch();
+}
+
+// The schedule scores between 1 and cap candidates; the slice count (and so
+// the partial-sum buffer) depends on the count, so size for the largest.
+size_t max_sre_workspace_bytes(int nh, int d, int cap) {
+    size_t m = 0;
+    for (int n = 1; n <= cap; ++n) {
+        const size_t b = sre_workspace_bytes(nh, 1, d, n);
+        if (b > m) m = b;
+    }
+    return m;
+}
+
+struct LolaWs {
+    void *ck[2], *cv[2];
+    int *cpos[2];
+    int *keep_idx;
+    void *sre_ws;
+    void *readout_ws;
+};
+
+LolaWs carve_lola(void *ws, int nh, int T, int d, int window, int cache, int dtype) {
+    const int cap = cache + window;
+    const size_t es = elem_size(dtype);
+    char *p = static_cast<char *>(ws);
+    LolaWs w;
+    for (int b = 0; b < 2; ++b) {
+        w.ck[b] = p;
+        p += align_up((size_t)nh * cap * d * es, 256);
+        w.cv[b] = p;
+        p += align_up((size_t)nh * cap * d * es, 256);
+        w.cpos[b] = reinterpret_cast<int *>(p);
+        p += align_up((size_t)nh * cap * sizeof(int), 256);
+    }
+    w.keep_idx = reinterpret_cast<int *>(p);
+    p += align_up((size_t)nh * cap * sizeof(int), 256);
+    w.sre_ws = p;
+    p += align_up(max_sre_workspace_bytes(nh, d, cap), 256);
+    w.readout_ws = p;
+    (void)T;
+    return w;
+}
+
+template <typename Tin>
+cudaError_t lola_impl(const Tin *q, const Tin *k, const Tin *v, int dtype, int nh, int T, int d,
+                      int window, int cache, float eps, float tau, float *o, float *Hst,
+                      float *s, int *kept_pos, void *ws, cudaStream_t stream) {
+    const int U = window, cap = cache + window, G = T / U;
+    LolaWs w = carve_lola(ws, nh, T, d, window, cache, dtype);
+    int cur = 0, nc = 0;
+    cudaError_t err;
+    for (int g = 0; g < G; ++g) {
+        err = readout_impl<Tin>(q, k, v, nh, T, d, g * U, U, g >= 1 ? U * (g - 1) : 0,
+                                static_cast<const Tin *>(w.ck[cur]),
+                                static_cast<const Tin *>(w.cv[cur]), nc, cap, Hst, s, eps, tau,
+                                o, w.readout_ws, stream);
+        if (err != cudaSuccess) return err;
+        if (g < 1) continue;
+        lola_append_kernel<Tin><<<nh, 256, 0, stream>>>(
+            k, v, T, d, U * (g - 1), U, static_cast<Tin *>(w.ck[cur]),
+            static_cast<Tin *>(w.cv[cur]), w.cpos[cur], cap, nc);
+        if ((err = after_launch()) != cudaSuccess) return err;
+        const int n = nc + U;
+        const int m = cache < n ? cache : n;
+        err = sre_impl<Tin>(Hst, s, static_cast<const Tin *>(w.ck[cur]),
+                            static_cast<const Tin *>(w.cv[cur]), w.cpos[cur], nh, d, n, cap,
+                            cache, eps, 1, nullptr, w.keep_idx, Hst, s, w.sre_ws, stream);
+        if (err != cudaSuccess) return err;
+        lola_compact_kernel<Tin><<<nh, 256, 0, stream>>>(
+            static_cast<const Tin *>(w.ck[cur]), static_cast<const Tin *>(w.cv[cur]),
+            w.cpos[cur], static_cast<Tin *>(w.ck[1 - cur]), static_cast<Tin *>(w.cv[1 - cur]),
+            w.cpos[1 - cur], w.keep_idx, m, cap, d,
+            kept_pos ? kept_pos + (size_t)(g - 1) * nh * cache : nullptr, cache);
+        if ((err = after_launch()) != cudaSuccess) return err;
+        cur = 1 - cur;
+        nc = m;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t sre_workspace_bytes(int B, int H, int d, int n_cand) {
+    const int nh = B * H;
+    return align_up(partial_floats(nh, n_cand, d) * sizeof(float), 256) +
+           align_up((size_t)nh * n_cand * sizeof(int), 256) +
+           align_up((size_t)nh * sizeof(int), 256);
+}
+
+size_t readout_workspace_bytes(int B, int H, int d, int nq) {
+    return align_up(partial_floats(B * H, nq, d) * sizeof(float), 256);
+}
+
+size_t lola_workspace_bytes(int B, int H, int T, int d, int window, int cache) {
+    const int nh = B * H, cap = cache + window;
+    const size_t es = 4;  // sized for the wider input type
+    size_t b = 0;
+    for (int i = 0; i < 2; ++i)
+        b += 2 * align_up((size_t)nh * cap * d * es, 256) +
+             align_up((size_t)nh * cap * sizeof(int), 256);
+    b += align_up((size_t)nh * cap * sizeof(int), 256);
+    b += align_up(max_sre_workspace_bytes(nh, d, cap), 256);
+    b += readout_workspace_bytes(nh, 1, d, window);
+    (void)T;
+    return b;
+}
+
+cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, const void *vc,
+                           const int *pos, int dtype, int B, int H, int d, int n_cand,
+                           int cand_stride, int keep, float eps, int merge, float *scores,
+                           int *keep_idx, float *Hst_mut, float *s_mut, void *ws,
+                           size_t ws_bytes, cudaStream_t stream) {
+    (void)ws_bytes;
+    const int nh = B * H;
+    if (dtype == 0)
+        return sre_impl<float>(Hst, s, static_cast<const float *>(kc),
+                               static_cast<const float *>(vc), pos, nh, d, n_cand, cand_stride,
+                               keep, eps, merge, scores, keep_idx, Hst_mut, s_mut, ws, stream);
+    return sre_impl<__nv_bfloat16>(Hst, s, static_cast<const __nv_bfloat16 *>(kc),
+                                   static_cast<const __nv_bfloat16 *>(vc), pos, nh, d, n_cand,
+                                   cand_stride, keep, eps, merge, scores, keep_idx, Hst_mut,
+                                   s_mut, ws, stream);
+}
+
+cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B,
+                           int H, int T, int d, int seg0, int nq, int w0, const void *ck,
+                           const void *cv, int nc, int cap, const float *Hst, const float *s,
+                           float eps, float tau, float *o, void *ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    (void)ws_bytes;
+    const int nh = B * H;
+    if (dtype == 0)
+        return readout_impl<float>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                   static_cast<const float *>(v), nh, T, d, seg0, nq, w0,
+                                   static_cast<const float *>(ck),
+                                   static_cast<const float *>(cv), nc, cap, Hst, s, eps, tau, o,
+                                   ws, stream);
+    using bf = __nv_bfloat16;
+    return readout_impl<bf>(static_cast<const bf *>(q), static_cast<const bf *>(k),
+                            static_cast<const bf *>(v), nh, T, d, seg0, nq, w0,
+                            static_cast<const bf *>(ck), static_cast<const bf *>(cv), nc, cap,
+                            Hst, s, eps, tau, o, ws, stream);
+}
+
+cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                     int T, int d, int window, int cache, float eps, float tau, float *o,
+                     float *Hst, float *s, int *kept_pos, void *ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+    (void)ws_bytes;
+    const int nh = B * H;
+    if (dtype == 0)
+        return lola_impl<float>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                static_cast<const float *>(v), dtype, nh, T, d, window, cache,
+                                eps, tau, o, Hst, s, kept_pos, ws, stream);
+    using bf = __nv_bfloat16;
+    return lola_impl<bf>(static_cast<const bf *>(q), static_cast<const bf *>(k),
+                         static_cast<const bf *>(v), dtype, nh, T, d, window, cache, eps, tau, o,
+                         Hst, s, kept_pos, ws, stream);
+}
+
+}  // namespace kata

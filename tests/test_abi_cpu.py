@@ -1,0 +1,110 @@
+"""The C-ABI library loads on a CPU-only host, exports every symbol the header
+declares, and rejects invalid arguments with a status before any launch."""
+import ctypes as C
+import re
+from pathlib import Path
+
+import pytest
+
+import kernelized_linear_attention_chunked_b200 as kata
+from kernelized_linear_attention_chunked_b200 import _binding
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "kata.h"
+
+
+def header_functions():
+    text = HEADER.read_text()
+    return re.findall(r"KATA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_symbols_exported_and_bound():
+    names = header_functions()
+    assert len(names) == 19
+    L = kata.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_binding.SIGNATURES)
+
+
+def test_header_argument_counts_match_binding():
+    text = HEADER.read_text()
+    for name, (_, args) in _binding.SIGNATURES.items():
+        m = re.search(r"KATA_API[^;(]*\b" + name + r"\(([^)]*)\)", text)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(args), name
+
+
+def test_status_strings_and_helpers():
+    L = kata.lib()
+    assert L.kata_version() >= 100
+    assert L.kata_status_string(0) == b"KATA_OK"
+    assert L.kata_status_string(4) == b"KATA_ERR_TIMEOUT"
+    assert L.kata_status_string(99) == b"KATA_ERR_UNKNOWN"
+    assert kata.launch_count() == 0  # validation failures launch nothing
+    for d in (16, 32, 64):
+        assert kata.packed_dim(d) == d * (d + 1) // 2
+
+
+def test_workspace_queries():
+    L = kata.lib()
+    assert L.kata_prefill_workspace_bytes(1, 1, 256, 16, 64, 0) > 0
+    assert L.kata_prefill_workspace_bytes(1, 1, 250, 16, 64, 0) == 0  # T not a multiple
+    assert L.kata_prefill_workspace_bytes(1, 1, 256, 24, 64, 0) == 0  # d not built
+    assert L.lola_sre_workspace_bytes(2, 8, 64, 192) > 0
+    assert L.lola_sre_workspace_bytes(2, 8, 64, 2000) == 0
+    assert L.lola_prefill_workspace_bytes(2, 8, 8192, 64, 64, 128) > 0
+    assert L.kata_prefill_path(1, 1, 256, 16, 64, 0) == 0  # fp32: CUDA cores
+    assert L.kata_prefill_path(1, 1, 250, 16, 64, 0) == -1
+    big = L.kata_prefill_host_workspace_bytes(1, 1, 256, 16, 64, 0)
+    assert big >= 4 * 256 * 16 * 4
+
+
+FAKE = C.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+MISALIGNED = C.c_void_p((1 << 20) + 4)
+
+
+def _prefill(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=0, B=1, H=1, T=256, d=16, chunk=64, eps=1e-6,
+             H_in=None, s_in=None, o=FAKE, H_out=None, s_out=None, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return kata.lib().kata_prefill(*a.values(), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1),
+    (dict(k=MISALIGNED), 1),
+    (dict(d=24), 2),
+    (dict(chunk=48), 2),
+    (dict(T=250), 1),
+    (dict(B=0), 1),
+    (dict(dtype=7), 2),
+    (dict(eps=-1.0), 1),
+    (dict(H_in=FAKE), 1),  # s_in missing
+    (dict(ws=None, ws_bytes=0), 5),
+])
+def test_prefill_validation(kw, status):
+    assert _prefill(**kw) == status
+    assert kata.lib().kata_last_error()
+
+
+def test_decode_and_lola_validation():
+    L = kata.lib()
+    assert L.kata_decode_step(FAKE, FAKE, FAKE, 1, 2, 2, 48, 1e-6, FAKE, FAKE, FAKE, None) == 2
+    assert L.kata_decode_step(FAKE, None, FAKE, 1, 2, 2, 64, 1e-6, FAKE, FAKE, FAKE, None) == 1
+    assert L.lola_sre_score_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 64, 0, 4, 1e-6, 0,
+                                 None, FAKE, None, None, FAKE, 1 << 30, None) == 1
+    assert L.lola_sre_score_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 64, 8, 4, 1e-6, 1,
+                                 None, FAKE, None, None, FAKE, 1 << 30, None) == 1
+    assert L.lola_hybrid_readout(FAKE, FAKE, FAKE, 1, 1, 1, 128, 64, 64, 64, 80, FAKE, FAKE, 0,
+                                 8, FAKE, FAKE, 1e-6, 0.125, FAKE, FAKE, 1 << 30, None) == 1
+    assert L.lola_prefill(FAKE, FAKE, FAKE, 1, 1, 1, 100, 64, 64, 8, 1e-6, 0.125, FAKE, FAKE,
+                          FAKE, None, FAKE, 1 << 30, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding, "LIB_PATH", tmp_path / "missing.so")
+    with pytest.raises(kata.KataError):
+        _binding.lib()
