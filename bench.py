@@ -147,21 +147,26 @@ def traffic_record(kernel: str, workload: str):
 
 # ---------------------------------------------------------------- oracle ----
 
-def cpu_baseline(w, max_heads: int | None = None):
+def cpu_baseline(w, max_heads: int | None = None, min_seconds: float = 0.0):
     """The fp64 oracle (recurrent form, the fastest exact CPU form) on a
-    bounded sample of the workload, scaled to tokens/s."""
+    bounded sample of the workload, scaled to tokens/s. The sample is
+    `max_heads` heads of the workload (all by default), repeated until
+    `min_seconds` of CPU time have passed."""
     import oracle
     q, k, v = prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed, recipe=w.recipe)
     nh = w.B * w.H if max_heads is None else min(max_heads, w.B * w.H)
     qf, kf, vf = (x.reshape(w.B * w.H, w.T, w.d)[:nh] for x in (q, k, v))
+    reps, dt = 0, 0.0
     t0 = time.perf_counter()
-    oracle.recurrent(qf, kf, vf, w.eps)
-    dt = time.perf_counter() - t0
-    tokens = w.T * nh / w.H  # a token is one position of one sequence (all heads)
+    while reps == 0 or dt < min_seconds:
+        oracle.recurrent(qf, kf, vf, w.eps)
+        reps += 1
+        dt = time.perf_counter() - t0
+    tokens = reps * w.T * nh / w.H  # a token is one position of one sequence (all heads)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"recurrent fp64 form over {nh} of {w.B * w.H} heads x {w.T} tokens "
-                      f"({dt:.2f} s)", "seconds": dt}
+            "sample": f"recurrent fp64 form, {nh} of {w.B * w.H} heads x {w.T} tokens, "
+                      f"{reps} repetition(s), {dt:.1f} s", "seconds": dt / reps}
 
 
 def run_reference(args, rank: int):
@@ -169,7 +174,7 @@ def run_reference(args, rank: int):
         return
     import oracle  # noqa: F401
     w = WORKLOADS[HEADLINE]
-    nh = 4  # a bounded sample per step: 4 of 32 heads (about a second of CPU work)
+    nh = 8  # a bounded sample per step: 8 of 32 heads
     for _ in range(args.warmup):
         cpu_baseline(w, max_heads=nh)
     times, vals = [], []
@@ -239,6 +244,27 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     peaks, peak_kind = load_peaks()
+    if args.only:
+        fn = {"decode": lambda: bench_decode(kata, args, dev, stream, peaks, dist_on, world),
+              "long_prefill": lambda: bench_long_prefill(kata, args, dev, stream, peaks,
+                                                         dist_on, world),
+              "lola": lambda: bench_lola(kata, args, dev, stream, dist_on, world)}[args.only]
+        res = fn()
+        if rank == 0:
+            print(json.dumps({"only": args.only, args.only: res}), flush=True)
+        return
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        line = run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind)
+    line["clocks"] = clocks.summary()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(WORKLOADS[HEADLINE], min_seconds=10.0)
+        cpu.pop("seconds")
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     w = WORKLOADS[HEADLINE]
 
     # Headline: prefill over resident inputs. The batch's inputs and outputs
@@ -262,11 +288,10 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
     kata.sync_status()
     barrier(dist_on)
     n0 = kata.launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clocks:
-        t0 = time.perf_counter()
-        ms = time_events(step, args.steps, stream)
-        barrier(dist_on)
-        wall = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    ms = time_events(step, args.steps, stream)
+    barrier(dist_on)
+    wall = time.perf_counter() - t0
     launches = kata.launch_count() - n0
     kata.sync_status()
     ms = max_over_ranks(ms, dist_on)
@@ -324,11 +349,6 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
         sub["long_prefill"] = bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world)
         sub["lola"] = bench_lola(kata, args, dev, stream, dist_on, world)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, max_heads=8)
-        cpu.pop("seconds")
-
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -340,11 +360,10 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
                              "> 126 MB L2)"},
             "prefill": {"tflops": tflops, "frac_bf16_peak": tflops / peaks["bf16_tflops"],
                         "peak_source": peak_kind},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clocks.summary(), "wall_s": wall}
+            "roofline": roof, "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches,
+            "wall_s": wall}
     line.update(sub)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    return line
 
 
 def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
@@ -441,6 +460,8 @@ def main():
     ap.add_argument("--impl", choices=["kata", "reference"], default="kata")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["decode", "long_prefill", "lola"], default=None,
+                    help="run one sub-benchmark alone (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
