@@ -182,6 +182,34 @@ KATA_API int lola_sre_score_topk(const float *Hst, const float *s, const void *k
                         float eps, int merge, float *scores, int *keep_idx, float *Hst_mut,
                         float *s_mut, void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * lola_sre_score_topk without a workspace argument. (The pages have no
+ * counterpart: this is a calling convenience of this library.)
+ *
+ * For callers that cannot allocate device memory when they score candidates,
+ * for example a serving loop whose memory pool is sized once and must not
+ * grow, or a host program with no device allocator of its own. The scratch
+ * the scoring needs comes from one fixed array of 8 MiB of device memory that
+ * the library holds on every GPU it is loaded on, until the process exits.
+ * This call allocates nothing.
+ *
+ * Arguments, results and errors are those of lola_sre_score_topk. Sizes whose
+ * scratch would exceed 8 MiB (lola_sre_workspace_bytes() > 8 MiB; for d = 64
+ * and 192 candidates, up to 33 heads B*H) return KATA_ERR_WORKSPACE with the
+ * numbers in kata_last_error().
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture. Every call
+ * shares the one array and it keeps what the last call left there (nothing in
+ * it needs to start at zero). Two calls whose kernels overlap on the GPU, from
+ * different streams or host threads, race on the array: serialise them.
+ */
+KATA_API int lola_sre_score_topk_noalloc(const float *Hst, const float *s, const void *kc,
+                                         const void *vc, const int *pos, int dtype, int B,
+                                         int H, int d, int n_cand, int keep, float eps,
+                                         int merge, float *scores, int *keep_idx,
+                                         float *Hst_mut, float *s_mut, void *stream);
+
 /* Device workspace bytes lola_hybrid_readout needs. */
 KATA_API size_t lola_readout_workspace_bytes(int B, int H, int d, int nq);
 

@@ -40,6 +40,8 @@ SIGNATURES = {
     "lola_sre_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "lola_sre_score_topk": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                                  _vp, _vp, _vp, _vp, _sz, _vp]),
+    "lola_sre_score_topk_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f,
+                                         _i, _vp, _vp, _vp, _vp, _vp]),
     "lola_readout_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "lola_hybrid_readout": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _i,
                                  _i, _vp, _vp, _f, _f, _vp, _vp, _sz, _vp]),

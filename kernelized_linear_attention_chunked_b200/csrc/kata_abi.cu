@@ -326,6 +326,43 @@ int lola_sre_score_topk(const float *Hst, const float *s, const void *kc, const 
     return KATA_OK;
 }
 
+int lola_sre_score_topk_noalloc(const float *Hst, const float *s, const void *kc,
+                                const void *vc, const int *pos, int dtype, int B, int H, int d,
+                                int n_cand, int keep, float eps, int merge, float *scores,
+                                int *keep_idx, float *Hst_mut, float *s_mut, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if (n_cand < 1 || n_cand > 1024)
+        return fail(KATA_ERR_INVALID_ARG, "n_cand=%d must be in [1, 1024]", n_cand);
+    if (keep < 0) return fail(KATA_ERR_INVALID_ARG, "keep=%d must be >= 0", keep);
+    if (merge != 0 && merge != 1) return fail(KATA_ERR_INVALID_ARG, "merge must be 0 or 1");
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_REQUIRE_PTR(kc);
+    KATA_REQUIRE_PTR(vc);
+    KATA_REQUIRE_PTR(pos);
+    KATA_OPTIONAL_PTR(scores);
+    if (keep > 0) KATA_REQUIRE_PTR(keep_idx);
+    if (merge) {
+        KATA_REQUIRE_PTR(Hst_mut);
+        KATA_REQUIRE_PTR(s_mut);
+    }
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t need = kata::sre_workspace_bytes(B, H, d, n_cand);
+    const size_t cap = kata::sre_noalloc_capacity();
+    if (need > cap)
+        return fail(KATA_ERR_WORKSPACE,
+                    "B=%d H=%d d=%d n_cand=%d needs %zu bytes of scratch but the fixed scratch "
+                    "holds %zu; call lola_sre_score_topk with a workspace instead",
+                    B, H, d, n_cand, need, cap);
+    cudaError_t e = kata::sre_score_topk_noalloc(Hst, s, kc, vc, pos, dtype, B, H, d, n_cand,
+                                                 keep, eps, merge, scores, keep_idx, Hst_mut,
+                                                 s_mut, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "lola_sre_score_topk_noalloc");
+    return KATA_OK;
+}
+
 size_t lola_readout_workspace_bytes(int B, int H, int d, int nq) {
     if (check_common(KATA_F32, B, H, d) || nq < 1 || nq > 256) return 0;
     return kata::readout_workspace_bytes(B, H, d, nq);

@@ -37,6 +37,14 @@ cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, con
                            int cand_stride, int keep, float eps, int merge, float *scores,
                            int *keep_idx, float *Hst_mut, float *s_mut, void *ws,
                            size_t ws_bytes, cudaStream_t stream);
+// Same as sre_score_topk with scratch in a fixed device array (no caller
+// workspace); sre_noalloc_capacity() is that array's size in bytes.
+size_t sre_noalloc_capacity();
+cudaError_t sre_score_topk_noalloc(const float *Hst, const float *s, const void *kc,
+                                   const void *vc, const int *pos, int dtype, int B, int H,
+                                   int d, int n_cand, int keep, float eps, int merge,
+                                   float *scores, int *keep_idx, float *Hst_mut, float *s_mut,
+                                   cudaStream_t stream);
 size_t readout_workspace_bytes(int B, int H, int d, int nq);
 cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B,
                            int H, int T, int d, int seg0, int nq, int w0, const void *ck,

@@ -23,6 +23,8 @@
 //  hybrid_finish  window + cache softmax terms, plus the state partials, one
 //                 shared denominator.
 //  append/compact the cache bookkeeping of the schedule.
+#include <mutex>
+
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
@@ -586,6 +588,69 @@ cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int
     return lola_impl<bf>(static_cast<const bf *>(q), static_cast<const bf *>(k),
                          static_cast<const bf *>(v), dtype, nh, T, d, window, cache, eps, tau, o,
                          Hst, s, kept_pos, ws, stream);
+}
+
+}  // namespace kata
+
+namespace kata {
+
+// ---------------------------------------------------------------------------
+// SRE scoring + top-k with a fixed scratch area instead of a caller workspace.
+//
+// Some callers cannot allocate device memory at the point where they score
+// candidates: code running under an allocator that must not grow (a serving
+// loop with a pre-sized memory pool), or a host program that has no allocator
+// of its own for device scratch. For them the scratch lives in one file-scope
+// device array of kNoAllocScratchBytes, created when the library is loaded on
+// a device and kept until the process exits.
+//
+// Set-up: the array's device address is looked up once per device, with that
+// device current, by the first call on that device. Make that first call
+// before any stream capture.
+// Sharing: every call uses the same array and it keeps the last call's
+// contents. Nothing in it needs to start at zero (every value the kernels read
+// is written earlier in the same call). Calls whose kernels overlap on the GPU
+// (other streams, other host threads) race on the array; serialise them.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[128] = {nullptr};
+
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t sre_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+cudaError_t sre_score_topk_noalloc(const float *Hst, const float *s, const void *kc,
+                                   const void *vc, const int *pos, int dtype, int B, int H,
+                                   int d, int n_cand, int keep, float eps, int merge,
+                                   float *scores, int *keep_idx, float *Hst_mut, float *s_mut,
+                                   cudaStream_t stream) {
+    void *scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    return sre_score_topk(Hst, s, kc, vc, pos, dtype, B, H, d, n_cand, n_cand, keep, eps,
+                          merge, scores, keep_idx, Hst_mut, s_mut, scratch,
+                          kNoAllocScratchBytes, stream);
 }
 
 }  // namespace kata
