@@ -69,7 +69,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 // Bounded wait: returns false (and records `code` in *err) if the phase with
 // this parity has not completed after `limit` polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
-                                          unsigned int code, uint32_t limit = 1u << 26) {
+                                          unsigned int code, uint32_t limit = 1u << 22) {
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (err && (i & 1023u) == 1023u && *((volatile unsigned int *)err) != 0u) return false;
@@ -80,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
 
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
                                                   unsigned int *err, unsigned int code,
-                                                  uint32_t limit = 1u << 26) {
+                                                  uint32_t limit = 1u << 22) {
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if (err && (i & 1023u) == 1023u && *((volatile unsigned int *)err) != 0u) return false;
