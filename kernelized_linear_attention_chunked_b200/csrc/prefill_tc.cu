@@ -1,43 +1,50 @@
-// Causal chunked prefill on the 5th-generation tensor cores (tcgen05).
+// Tensor-core (tcgen05) chunked prefill for bf16 inputs, d = 32 or 64.
 //
-// "Kernelized Linear Attention: Breaking the Capacity Wall with Symmetric
-// Cones", s2.3: inside a chunk the work runs on tensor cores, the state is
-// carried across chunks, and the chunked state form is exact. With the
-// feature of s2.2 (phi(x) = x x^T), for chunk c of 128 tokens:
-//   O_c   = (S (.) S (.) M) V_c + Phi(Q_c) H_{c-1}      S = Q_c K_c^T, M causal
-//   z_c   = rowsum(S (.) S (.) M) + q^T G_{c-1} q       G = sum_j k_j k_j^T
-//   o     = O_c / (z_c + eps)
-//   H_c   = H_{c-1} + Phi(K_c)^T V_c,   G_c = G_{c-1} + K_c^T K_c
-// (phi(q)^T s = q^T G q, so the normaliser state is the d x d matrix G.)
+// What it computes ("Kernelized Linear Attention: Breaking the Capacity Wall
+// with Symmetric Cones", technical summary §2.2 rank-one PSD cone and §2.3
+// chunked parallelism with the exact chunked state form):
 //
-// Design (one cluster of kNC CTAs per (batch, head)):
-//  - The packed dimension D = d(d+1)/2 is cut into 128-row tiles; rank 0 owns
-//    a few tiles plus the intra-chunk part and G, ranks 1.. own the rest.
-//    Every tile's fp32 state H_i (128 x d) lives in tensor memory for the whole
-//    sequence.
-//  - Internally the state is kept without the sqrt(2) of the packed layout:
-//    row (a, b) holds sum_j k_a k_b v_j; the readout multiplies off-diagonal
-//    rows by 2 (folded into Phi(Q), exact in bf16). H_in / H_out are converted
-//    to and from the packed layout of include/kata.h at the edges.
-//  - Phi(K_c)^T (A operand of the state update, lane = packed row) and
-//    Phi(Q_c) (A operand of the readout, lane = query) are generated by 8
-//    worker warps straight into tensor-memory A slots (bf16x2 products), so
-//    the tensor core reads only the B operands from shared memory.
-//  - The readout's B operand is a bf16 copy of the state tile ("mirror"),
-//    converted by the workers one tile ahead of the MMA into a 2-slot ring.
-//  - Per chunk each CTA holds a partial O (128 x d, fp32). Row quarter qb is
-//    owned by CTA qb % kNC; the other CTAs store their partial rows into the
-//    owner's shared memory (DSMEM) and arrive on its barrier; the owner adds
-//    them one chunk later (so nobody waits), divides and writes o.
-//  - Q, K, V chunks arrive by TMA (128-byte swizzle) in a 2-stage ring; one
-//    thread issues every MMA; all waits are bounded and report through the
-//    per-device error word.
+//   o_i = phi(q_i)^T H_i / (phi(q_i)^T s_i + eps),   H_i = sum_{j<=i} phi(k_j) v_j^T,
+//   s_i = sum_{j<=i} phi(k_j),   <phi(q), phi(k)> = (q.k)^2.
+//
+// Two kernels, split along the dependency structure of the chunked form:
+//
+//  1. state_kernel — the carry across chunks (§2.3's inter-chunk state
+//     propagation). One CTA owns one 128-row tile of the feature space of one
+//     head and walks the sequence chunk by chunk (128 tokens), accumulating
+//     dH = Phi(K_c)^T [V_c | 1] on the tensor cores into fp32 tensor memory.
+//     Every L tokens it writes the exclusive prefix state (the state before
+//     the interval) as a bf16 snapshot laid out as the readout's MMA operand.
+//     Feature rows are independent, so a head's tiles run as separate CTAs
+//     with no communication.
+//  2. readout_kernel — fully parallel over (head, 128-query tile):
+//       inter part  Phi(Q) [H | s](snapshot at the start of the interval),
+//       intra part  ((Q K^T)^2 masked causally) [V | 1] over the keys from
+//                   the interval start to the query (the quadratic form),
+//     both accumulated in one fp32 tensor-memory tile, then normalised.
+//
+// Feature space. phi(x) x phi(y) = (x.y)^2 is expanded over 8x8 blocks of the
+// outer product x x^T: an off-diagonal block (A < B) holds x_a x_b for a in
+// block A, b in block B (each unordered pair once, weight 2 on the query side);
+// a diagonal block (A, A) holds all 64 ordered products (weight 1, so a pair
+// a != b inside it counts twice, a = b once). Every block is one 64-feature
+// slice: d = 32 has 10 slices, d = 64 has 36. The state is stored without the
+// sqrt(2) of the canonical packed layout; kata_prefill's H_in/H_out use the
+// canonical one and the state kernel converts at both ends.
+//
+// Column layout of the fp32 accumulators (state and output): columns 0..d-1
+// hold H (or the numerator), columns 64..79 all hold s (or the denominator)
+// because the [V | 1] operand is the V tile followed by a 64-wide all-ones
+// block; for d = 32 columns 32..63 are zero. The snapshot slices hold rows
+// 0..d-1 = H and d..d+15 = s, so the inter MMA writes the denominator part to
+// column d: the readout sums columns d and 64 (the same column for d = 64).
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
+#include <stdint.h>
 
 #include <mutex>
-#include <utility>
 
-#include "kata_common.cuh"
 #include "kata_internal.h"
 #include "sm100.cuh"
 
@@ -46,778 +53,680 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kC = 128;         // tokens per chunk (MMA M)
-constexpr int kNC = 4;          // CTAs per cluster (per head)
-constexpr int kWorkers = 8;     // worker warps
-constexpr int kThreads = 32 * (2 + kWorkers);
-constexpr int kKtPitch = 272;   // bytes per row of the transposed K tile
-
-// ---------------------------------------------------------------------------
-// Internal order of the packed rows: for every a, the run (a, b) with b from a
-// (a even) or a+1 (a odd) to d-1, each run of even length; then the odd
-// diagonals (1,1), (3,3), ... Consecutive rows (2m, 2m+1) share a and have an
-// even b, so one bf16x2 product yields both.
-// Code: bits 0-7 b, 8-15 a, 16-17 kind (0 pair, 1 odd-diagonal pair, 2 pad).
-__host__ __device__ constexpr uint32_t row_code(int d, int r) {
-    int n = 0;
-    for (int a = 0; a < d; ++a) {
-        const int b0 = (a & 1) ? a + 1 : a;
-        const int len = d - b0;
-        if (r < n + len) return (uint32_t)((a << 8) | (b0 + (r - n)));
-        n += len;
-    }
-    const int k = r - n;
-    if (k < d / 2) {
-        const int a = 2 * k + 1;
-        return (uint32_t)((1u << 16) | (a << 8) | a);
-    }
-    return 2u << 16;
-}
-
-__host__ __device__ constexpr int canon_index(int d, int a, int b) {
-    return a * d - a * (a - 1) / 2 + (b - a);
-}
-
-// ---------------------------------------------------------------- Phi(Q) ---
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t x, uint32_t y) {
-    __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&x),
-                               *reinterpret_cast<__nv_bfloat162 *>(&y));
-    return *reinterpret_cast<uint32_t *>(&r);
-}
-
-constexpr uint32_t kBf16One = 0x3F80u, kBf16Two = 0x4000u;
-
-// Packed column COL of Phi(Q) for one query held in R (R[i] = q_{2i}, q_{2i+1}):
-// rows (2 COL, 2 COL + 1) of the internal order, weighted by w^2 (1 on the
-// diagonal, 2 off it).
-template <int DH, int COL>
-__device__ __forceinline__ uint32_t q_column(const uint32_t (&R)[32]) {
-    constexpr uint32_t code = row_code(DH, 2 * COL);
-    constexpr uint32_t kind = code >> 16;
-    constexpr int a = (code >> 8) & 255, b = code & 255;
-    if constexpr (kind == 2) {
-        return 0u;
-    } else if constexpr (kind == 1) {  // (a, a), (a + 2, a + 2), a odd
-        const uint32_t y = __byte_perm(R[a / 2], R[(a + 2) / 2], 0x7632);
-        return hmul2(y, y);
-    } else {
-        const uint32_t qa = __byte_perm(R[a / 2], 0u, (a & 1) ? 0x3232 : 0x1010);
-        constexpr uint32_t w = (a == b) ? (kBf16One | (kBf16Two << 16))
-                                        : (kBf16Two | (kBf16Two << 16));
-        return hmul2(hmul2(qa, w), R[b / 2]);
-    }
-}
-
-template <int DH, int COL0, int... I>
-__device__ __forceinline__ void q_columns16(const uint32_t (&R)[32], uint32_t (&out)[16],
-                                            std::integer_sequence<int, I...>) {
-    ((out[I] = q_column<DH, COL0 + I>(R)), ...);
-}
-
-// 16 packed columns starting at COL0, for every COL0 = 16 m a worker can need.
-template <int DH, int M>
-__device__ __forceinline__ void q_block(const uint32_t (&R)[32], uint32_t (&out)[16]) {
-    q_columns16<DH, 16 * M>(R, out, std::make_integer_sequence<int, 16>{});
-}
-
-template <int DH, int... M>
-__device__ __forceinline__ void q_dispatch(int m, const uint32_t (&R)[32], uint32_t (&out)[16],
-                                           std::integer_sequence<int, M...>) {
-    ((m == M ? (q_block<DH, M>(R, out), 0) : 0), ...);
-}
-
-// ------------------------------------------------------------ parameters ---
-
-struct TcParams {
-    int T, nch;             // tokens, chunks of kC
-    int nheads;
-    float eps;
-    int tile_begin[kNC + 1];
-    const float *H_in, *s_in;
-    float *o, *H_out, *s_out;
-    unsigned int *err;
-};
+constexpr int kTile = 128;         // tokens per chunk / query tile; rows per state tile
+constexpr int kTileBytes = 16384;  // one 128 x 64 bf16 tile, 128-byte swizzle
+constexpr int kAccCols = 80;       // accumulator columns: H (<= 64) | s x 16
+constexpr int kSCol = 64;          // first accumulator column holding s
+constexpr int kKtPitch = 272;      // bytes per row of the transposed K tile (256 + 16)
+constexpr int kWorkers = 128;      // 4 warps: one thread per tensor-memory lane
+constexpr int kThreads = 192;      // + MMA issuer warp + TMA producer warp
+constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
 
 template <int DH>
-struct Layout {
-    static constexpr int D = DH * (DH + 1) / 2;
-    static constexpr int NT = (D + 127) / 128;
-    static constexpr int PAY = DH / 2 + 4;                 // floats per (lane, half) payload
-    static constexpr uint32_t kQ = 16384, kK = 16384, kV = 128 * DH * 2;
-    static constexpr uint32_t kStage = kK + kQ + kV;       // K | Q | V
-    static constexpr uint32_t kStages = 2 * kStage;
-    static constexpr uint32_t kKt = 64 * kKtPitch;
-    static constexpr uint32_t kMirror = 128 * DH * 2;
-    static constexpr uint32_t kGm = 64 * 128;
-    static constexpr uint32_t kRecvOne = 2 * 32 * PAY * 4;      // one source, both halves
-    static constexpr uint32_t kRecv = 2 * (4 / kNC) * (kNC - 1) * kRecvOne;
-    static constexpr uint32_t oKt = kStages;
-    static constexpr uint32_t oMirror = (oKt + kKt + 1023) / 1024 * 1024;
-    static constexpr uint32_t oGm = oMirror + 2 * kMirror;
-    static constexpr uint32_t oRecv = oGm + kGm;
-    static constexpr uint32_t oZ = oRecv + kRecv;               // z exchange [2][128] fp32
-    static constexpr uint32_t oTab = oZ + 2 * 128 * 4;          // row codes [NT*128] u32
-    static constexpr uint32_t oBar = (oTab + NT * 128 * 4 + 15) / 16 * 16;
-    static constexpr uint32_t kBars = 64;
-    static constexpr uint32_t oTmemSlot = oBar + kBars * 8;
-    static constexpr uint32_t kBytes = oTmemSlot + 16 + 1024;   // + alignment slack
-    static constexpr uint32_t kVsw = DH == 64 ? 128 : 64;       // V / mirror row bytes
-    static constexpr uint32_t kVsbo = 8 * kVsw;                 // 8-row group stride
-    static constexpr uint32_t kVlayout = DH == 64 ? 2u : 4u;    // 128B or 64B swizzle
+struct Shape {
+    static constexpr int NB = DH / 8;            // 8-wide index blocks
+    static constexpr int NS = NB * (NB + 1) / 2;  // 64-feature slices
+    static constexpr int NT = (NS + 1) / 2;       // 128-row state tiles
+    static constexpr int NSNAP = DH + 16;         // snapshot rows: H | s x 16
+    static constexpr int SLICE_BYTES = NSNAP * 128;
 };
 
-// Barrier indices.
-enum : int {
-    kBarFull = 0,       // [2] TMA stage full
-    kBarEmpty = 2,      // [2] TMA stage empty
-    kBarAqReady = 4,    // [2]
-    kBarAqFree = 6,     // [2]
-    kBarAkReady = 8,    // [2]
-    kBarAkFree = 10,    // [2]
-    kBarMrReady = 12,   // [2]
-    kBarMrFree = 14,    // [2]
-    kBarOReady = 16,
-    kBarOFree = 17,
-    kBarSReady = 18,
-    kBarSUsed = 19,
-    kBarPReady = 20,
-    kBarPFree = 21,
-    kBarGReady = 22,
-    kBarGmReady = 23,
-    kBarFinal = 24,
-    kBarRecv = 25,      // [2] parity
-    kBarSendFree = 27,  // [2 parities][4 row quarters]
-    kBarKtReady = 35,   // transposed K written (all workers)
-    kBarKtFree = 36,    // transposed K no longer read (all workers)
-    kBarState = 40,     // [NT] state tile done (<= 17)
-};
-
-// Swizzled byte offset of 16-byte chunk `chunk` of row `row`, for rows of
-// `rowbytes` (128: 128-byte swizzle, 64: 64-byte swizzle).
-__device__ __forceinline__ uint32_t sw_off(uint32_t rowbytes, int row, int chunk) {
-    if (rowbytes == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
-    return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
+// Block pair (A, B), A <= B, of slice s: slices run A-major, B ascending.
+__device__ __forceinline__ void slice_blocks(int s, int nb, int &A, int &B) {
+    A = 0;
+    while (s >= nb - A) {
+        s -= nb - A;
+        ++A;
+    }
+    B = A + s;
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
+// Canonical packed index of the unordered pair {a, b} (upper triangle, a-major).
+__device__ __forceinline__ int canon_index(int a, int b, int d) {
+    const int lo = a < b ? a : b, hi = a < b ? b : a;
+    return lo * d - lo * (lo - 1) / 2 + (hi - lo);
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t x, uint32_t y) {
     uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
     return r;
 }
 
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-                 ::: "memory");
+__device__ __forceinline__ uint32_t bcast_lo(uint32_t x) { return (x & 0xFFFFu) * 0x10001u; }
+__device__ __forceinline__ uint32_t bcast_hi(uint32_t x) { return (x >> 16) * 0x10001u; }
+
+__device__ __forceinline__ void worker_sync() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kWorkers) : "memory");
 }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+// Element offset of 16-byte chunk `c` of row `r` in a tile with 128-byte rows
+// and the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c) {
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// Worker-warp wait: lane 0 polls (bounded), the verdict is broadcast, and
-// __syncwarp orders the other lanes' later accesses after lane 0's acquire.
+// One warp-uniform wait: lane 0 polls, the result is broadcast.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
-                                          unsigned int code, bool cluster_scope = false) {
+                                          unsigned int code) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0)
-        ok = cluster_scope ? mbar_wait_cluster(bar, parity, err, code) : mbar_wait(bar, parity, err, code);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     return ok != 0;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t local_addr, uint32_t cta, float a,
-                                              float b, float c, float d) {
-    asm volatile(
-        "{\n\t.reg .b32 ra;\n\t"
-        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "st.shared::cluster.v4.f32 [ra], {%2, %3, %4, %5};\n\t}" ::"r"(local_addr),
-        "r"(cta), "f"(a), "f"(b), "f"(c), "f"(d)
-        : "memory");
+__device__ __forceinline__ void tmem_ld16_f(uint32_t taddr, float (&f)[16]) {
+    uint32_t r[16];
+    tmem_ld16(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[e]);
 }
 
-template <int DH>
-__global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const TcParams p) {
-    using L = Layout<DH>;
-    constexpr int D = L::D;
-    constexpr int HALF = DH / 2;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::oBar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::oTmemSlot);
-    uint32_t *tab = reinterpret_cast<uint32_t *>(smem + L::oTab);
+// MN-major [V | 1] operand for 16 tokens starting at row `row0` of the V tile:
+// the V tile (64 bf16 per row, zero-filled past d) is the first 64-column
+// atom, the all-ones tile the second, `ones - v` bytes further on.
+__device__ __forceinline__ uint64_t vones_desc(uint32_t v, uint32_t ones, int row0) {
+    return smem_desc(v + row0 * 128, ones - v, 1024, kSwizzle128);
+}
 
+// K-major operand: 128-byte rows, 16 K-elements at byte offset 32 * kk.
+__device__ __forceinline__ uint64_t kmaj_desc(uint32_t base, int kk) {
+    return smem_desc(base + 32 * kk, 16, 1024, kSwizzle128);
+}
+
+// ---------------------------------------------------------------------------
+// State kernel
+// ---------------------------------------------------------------------------
+
+struct StateParams {
+    int nch;        // chunks per head
+    int cpi;        // chunks per snapshot interval
+    int nint;       // snapshot intervals per head
+    const float *H_in, *s_in;
+    float *H_out, *s_out;
+    uint8_t *snap;  // [heads][nint][NS][NSNAP][128 B]
+    unsigned int *err;
+};
+
+enum StateBar {
+    kSbKFull = 0,     // 2: K tile landed
+    kSbKFree = 2,     // 2: the workers transposed it (4 warp arrivals)
+    kSbVFull = 4,     // 2: V tile landed
+    kSbVFree = 6,     // 2: the chunk's MMAs finished reading it
+    kSbAFull = 8,     // 2: Phi(K)^T tile written to tensor memory (4 warp arrivals)
+    kSbDone = 10,     // 2: the MMAs of the chunk that used this A slot completed
+    kSbSnap = 12,     // the workers read the accumulator at an interval end (4 warp arrivals)
+    kSbCount = 13
+};
+
+template <int DH>
+struct StateSmem {
+    static constexpr int K0 = 0;                      // 2 x K tile
+    static constexpr int V0 = 2 * kTileBytes;         // 2 x V tile
+    static constexpr int ONES = 4 * kTileBytes;       // all-ones atom
+    static constexpr int KT = 5 * kTileBytes;         // K^T, DH rows of kKtPitch bytes
+    static constexpr int BAR = KT + DH * kKtPitch;    // barriers
+    static constexpr int SLOT = BAR + kSbCount * 8;   // tensor-memory base address
+    static constexpr int BYTES = SLOT + 16 + 1024;    // + alignment slack
+};
+
+// Tensor-memory columns of the state kernel (256 allocated): the fp32
+// accumulator and two Phi(K)^T slots (128 tokens as bf16 pairs each).
+constexpr uint32_t kStAcc = 0, kStA = 128;
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 2)
+    state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                 StateParams p) {
+    using S = Shape<DH>;
+    using L = StateSmem<DH>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();
-    const int bh = blockIdx.y;
-    const int tb0 = p.tile_begin[rank], nt = p.tile_begin[rank + 1] - tb0;
-    const bool lead = rank == 0;
+    const int tile = blockIdx.x, head = blockIdx.y;
     unsigned int *err = p.err;
 
-    // tensor-memory columns
-    const uint32_t cO = nt * DH, cAq = cO + DH, cAk = cAq + 64, cS = cAk + 64, cG = cS + 128;
-
-    // ---- set-up -------------------------------------------------------
-    for (int r = threadIdx.x; r < L::NT * 128; r += kThreads) tab[r] = row_code(DH, r);
     if (threadIdx.x == 0) {
-        mbar_init(&bar[kBarFull + 0], 1);
-        mbar_init(&bar[kBarFull + 1], 1);
-        mbar_init(&bar[kBarEmpty + 0], 1 + kWorkers);
-        mbar_init(&bar[kBarEmpty + 1], 1 + kWorkers);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[kBarAqReady + s], kWorkers);
-            mbar_init(&bar[kBarAqFree + s], 1);
-            mbar_init(&bar[kBarAkReady + s], kWorkers);
-            mbar_init(&bar[kBarAkFree + s], 1);
-            mbar_init(&bar[kBarMrReady + s], kWorkers);
-            mbar_init(&bar[kBarMrFree + s], 1);
-            mbar_init(&bar[kBarRecv + s], (kNC - 1) * 64 * (4 / kNC));
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar[kSbKFull + i], 1);
+            mbar_init(&bar[kSbKFree + i], 4);
+            mbar_init(&bar[kSbVFull + i], 1);
+            mbar_init(&bar[kSbVFree + i], 1);
+            mbar_init(&bar[kSbAFull + i], 4);
+            mbar_init(&bar[kSbDone + i], 1);
         }
-        mbar_init(&bar[kBarOReady], 1);
-        mbar_init(&bar[kBarOFree], kWorkers);
-        mbar_init(&bar[kBarSReady], 1);
-        mbar_init(&bar[kBarSUsed], kWorkers);
-        mbar_init(&bar[kBarPReady], 1);
-        mbar_init(&bar[kBarPFree], kWorkers);
-        mbar_init(&bar[kBarGReady], 1);
-        mbar_init(&bar[kBarGmReady], 4);
-        mbar_init(&bar[kBarFinal], 1);
-        for (int q = 0; q < 8; ++q) mbar_init(&bar[kBarSendFree + q], 2);
-        mbar_init(&bar[kBarKtReady], kWorkers);
-        mbar_init(&bar[kBarKtFree], kWorkers);
-        for (int i = 0; i < L::NT; ++i) mbar_init(&bar[kBarState + i], 1);
+        mbar_init(&bar[kSbSnap], 4);
         fence_barrier_init();
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
+    if (warp == 4) {
+        tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-    }
-    tc_fence_before();
-    cluster_sync();  // barriers of every CTA initialised before any remote arrive
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    const size_t row0 = (size_t)bh * p.T;  // first token row of this head
-
-    if (warp == 0) {
-        // ================================================== TMA producer ==
-        if (lane == 0) {
-            for (int c = 0; c < p.nch; ++c) {
-                const int s = c & 1;
-                if (c >= 2 && !mbar_wait(&bar[kBarEmpty + s], ((c >> 1) - 1) & 1, err, 0x101)) break;
-                uint8_t *st = smem + s * L::kStage;
-                mbar_arrive_expect_tx(&bar[kBarFull + s], L::kStage);
-                const int y = (int)(row0 + (size_t)c * kC);
-                tma_load_2d(st, &tmK, 0, y, &bar[kBarFull + s]);
-                tma_load_2d(st + L::kK, &tmQ, 0, y, &bar[kBarFull + s]);
-                tma_load_2d(st + L::kK + L::kQ, &tmV, 0, y, &bar[kBarFull + s]);
-            }
-            // drain: wait until the last loads have landed before teardown
-            for (int c = p.nch - 2; c < p.nch; ++c)
-                if (c >= 0) mbar_wait(&bar[kBarFull + (c & 1)], (c >> 1) & 1, err, 0x102);
-        }
-    } else if (warp == 1) {
-        // ===================================================== MMA issuer ==
-        if (lane == 0) {
-            const uint32_t i_tsv = idesc_bf16(128, DH, 0, 1);
-            const uint32_t i_s = idesc_bf16(128, 128, 0, 0);
-            const uint32_t i_g = idesc_bf16(128, 64, 1, 1);
-            const uint32_t i_p = idesc_bf16(128, 64, 0, 1);
-            uint32_t aq = 0, ak = 0, mr = 0;
-            const uint32_t gm_addr = smem_u32(smem + L::oGm);
-            for (int c = 0; c < p.nch; ++c) {
-                const int s = c & 1;
-                if (!mbar_wait(&bar[kBarFull + s], (c >> 1) & 1, err, 0x201)) break;
-                tc_fence_after();
-                const uint32_t kA = smem_u32(smem + s * L::kStage);
-                const uint32_t qA = kA + L::kK, vA = qA + L::kQ;
-                bool ok = true;
-                uint32_t o_acc = 0;
-                if (lead) {
-                    // S = Q K^T (both K-major, 128-byte swizzle)
-                    if (c >= 1) ok = ok && mbar_wait(&bar[kBarPFree], (c - 1) & 1, err, 0x202);
-                    tc_fence_after();
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + cS, smem_desc(qA + kk * 32, 16, 1024, kSwizzle128),
-                               smem_desc(kA + kk * 32, 16, 1024, kSwizzle128), i_s, kk > 0);
-                    mma_commit(&bar[kBarSReady]);
-                    // G += [K^T; Q^T] K (A, B MN-major; the Q^T rows are discarded)
-                    ok = ok && mbar_wait(&bar[kBarGmReady], c & 1, err, 0x203);
-                    tc_fence_after();
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + cG, smem_desc(kA + kk * 2048, L::kK, 1024, kSwizzle128),
-                               smem_desc(kA + kk * 2048, 16, 1024, kSwizzle128), i_g, 1);
-                    mma_commit(&bar[kBarGReady]);
-                }
-                if (c >= 1) ok = ok && mbar_wait(&bar[kBarOFree], (c - 1) & 1, err, 0x204);
-                tc_fence_after();
-                if (lead) {  // intra-chunk: O = (S^2 masked) V, two 64-token halves
-                    for (int h = 0; h < 2 && ok; ++h, ++aq) {
-                        const int sl = aq & 1;
-                        ok = mbar_wait(&bar[kBarAqReady + sl], (aq >> 1) & 1, err, 0x205);
-                        tc_fence_after();
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + cO, tmem + cAq + 32 * sl + 8 * kk,
-                                   smem_desc(vA + (4 * h + kk) * 16 * L::kVsw, 16, L::kVsbo,
-                                             L::kVlayout),
-                                   i_tsv, o_acc++ > 0);
-                        mma_commit(&bar[kBarAqFree + sl]);
-                    }
-                    // P = Q G_{c-1} into the S columns, once S has been read
-                    ok = ok && mbar_wait(&bar[kBarSUsed], c & 1, err, 0x206);
-                    tc_fence_after();
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + cS, smem_desc(qA + kk * 32, 16, 1024, kSwizzle128),
-                               smem_desc(gm_addr + kk * 2048, 16, 1024, kSwizzle128), i_p,
-                               kk > 0);
-                    mma_commit(&bar[kBarPReady]);
-                }
-                for (int i = 0; i < nt && ok; ++i) {
-                    // readout: O += Phi(Q)[:, tile i] * mirror_i
-                    const int ms = mr & 1;
-                    ok = mbar_wait(&bar[kBarMrReady + ms], (mr >> 1) & 1, err, 0x207);
-                    const uint32_t mA = smem_u32(smem + L::oMirror + ms * L::kMirror);
-                    for (int h = 0; h < 2 && ok; ++h, ++aq) {
-                        const int sl = aq & 1;
-                        ok = mbar_wait(&bar[kBarAqReady + sl], (aq >> 1) & 1, err, 0x208);
-                        tc_fence_after();
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + cO, tmem + cAq + 32 * sl + 8 * kk,
-                                   smem_desc(mA + (4 * h + kk) * 16 * L::kVsw, 16, L::kVsbo,
-                                             L::kVlayout),
-                                   i_tsv, o_acc++ > 0);
-                        mma_commit(&bar[kBarAqFree + sl]);
-                    }
-                    mma_commit(&bar[kBarMrFree + ms]);
-                    ++mr;
-                    // state update: H_i += Phi(K)^T[tile i, :] * V
-                    for (int h = 0; h < 2 && ok; ++h, ++ak) {
-                        const int sl = ak & 1;
-                        ok = mbar_wait(&bar[kBarAkReady + sl], (ak >> 1) & 1, err, 0x209);
-                        tc_fence_after();
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + i * DH, tmem + cAk + 32 * sl + 8 * kk,
-                                   smem_desc(vA + (4 * h + kk) * 16 * L::kVsw, 16, L::kVsbo,
-                                             L::kVlayout),
-                                   i_tsv, 1);
-                        mma_commit(&bar[kBarAkFree + sl]);
-                    }
-                    mma_commit(&bar[kBarState + i]);
-                }
-                mma_commit(&bar[kBarOReady]);
-                mma_commit(&bar[kBarEmpty + s]);
-                if (!ok) break;
-            }
-            mma_commit(&bar[kBarFinal]);
-        }
-    } else {
-        // ======================================================== workers ==
-        const int wi = warp - 2;
-        const int qtr = warp & 3;         // tensor-memory lane quarter
-        const int j = wi >> 2;            // half of the columns / tokens
-        const uint32_t lane_base = (uint32_t)(32 * qtr) << 16;
-        const int row = 32 * qtr + lane;  // query row / packed row in a tile / G row
-        uint8_t *kt = smem + L::oKt;
-        const uint32_t owner = qtr % kNC;
-        const bool own = owner == rank;
-        float *recv = reinterpret_cast<float *>(smem + L::oRecv);
-        uint32_t aq = 0, ak = 0, mr = 0;
-        bool ok = true;
-        float held[HALF];                 // owner: own partial of the previous chunk
-        float zheld = 0.f;
-        int held_c = -1;
-
-        // initial state: H_in (packed, with sqrt 2) -> internal rows (without)
-        for (int i = 0; i < nt; ++i) {
-            const uint32_t code = tab[(tb0 + i) * 128 + row];
-            const int a = (code >> 8) & 255, b = code & 255;
-            const bool pad = (code >> 16) == 2;
-            const int cr = pad ? 0 : canon_index(DH, a, b);
-            const float inv_w = (a == b) ? 1.f : 0.70710678118654752f;
-            for (int c0 = 0; c0 < HALF; c0 += 16) {
-                uint32_t r[16];
-                for (int e = 0; e < 16; ++e) {
-                    float x = 0.f;
-                    if (p.H_in && !pad)
-                        x = p.H_in[((size_t)bh * D + cr) * DH + j * HALF + c0 + e] * inv_w;
-                    r[e] = __float_as_uint(x);
-                }
-                tmem_st16(tmem + lane_base + i * DH + j * HALF + c0, r);
-            }
-        }
-        if (lead && qtr < 2) {  // G rows 0..63 from s_in; rows 64..127 zero
-            for (int c0 = 0; c0 < 32; c0 += 16) {
-                uint32_t r[16];
-                for (int e = 0; e < 16; ++e) {
-                    const int b = j * 32 + c0 + e, a = row;
-                    float x = 0.f;
-                    if (p.s_in && a < DH && b < DH) {
-                        const int lo = a < b ? a : b, hi = a < b ? b : a;
-                        x = p.s_in[(size_t)bh * D + canon_index(DH, lo, hi)] *
-                            (lo == hi ? 1.f : 0.70710678118654752f);
-                    }
-                    r[e] = __float_as_uint(x);
-                }
-                tmem_st16(tmem + lane_base + cG + j * 32 + c0, r);
-            }
-        } else if (lead) {
-            uint32_t r[16];
-            for (int e = 0; e < 16; ++e) r[e] = 0u;
-            for (int c0 = 0; c0 < 32; c0 += 16) tmem_st16(tmem + lane_base + cG + j * 32 + c0, r);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar(1, 32 * kWorkers);
-        tc_fence_after();
-
-        // mirror of the G rows for P = Q G (rank 0, rows 0..63 = quarters 0, 1)
-        auto g_to_mirror = [&]() {
-            if (qtr < 2) {
-                uint32_t r[16];
-                uint8_t *gm = smem + L::oGm;
-                for (int c0 = 0; c0 < 32; c0 += 16) {
-                    tmem_ld16(tmem + lane_base + cG + j * 32 + c0, r);
-                    tmem_ld_wait();
-                    for (int k = 0; k < 2; ++k) {  // two 16-byte chunks of 8 columns
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]), __uint_as_float(r[8 * k + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]), __uint_as_float(r[8 * k + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]), __uint_as_float(r[8 * k + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]), __uint_as_float(r[8 * k + 7]));
-                        const int chunk = (j * 32 + c0) / 8 + k;
-                        *reinterpret_cast<uint4 *>(gm + sw_off(128, row, chunk)) = v;
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBarGmReady]);
-            }
-        };
-        if (lead) g_to_mirror();
-
-        // mirror of state tile i (lane = packed row) into ring slot ms
-        auto state_to_mirror = [&](int i, int ms) {
-            uint8_t *m = smem + L::oMirror + ms * L::kMirror;
-            uint32_t r[16];
-            for (int c0 = 0; c0 < HALF; c0 += 16) {
-                tmem_ld16(tmem + lane_base + i * DH + j * HALF + c0, r);
-                tmem_ld_wait();
-                for (int k = 0; k < 2; ++k) {
-                    uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]), __uint_as_float(r[8 * k + 1]));
-                    v.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]), __uint_as_float(r[8 * k + 3]));
-                    v.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]), __uint_as_float(r[8 * k + 5]));
-                    v.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]), __uint_as_float(r[8 * k + 7]));
-                    const int chunk = (j * HALF + c0) / 8 + k;
-                    *reinterpret_cast<uint4 *>(m + sw_off(L::kVsw, row, chunk)) = v;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kBarMrReady + ms]);
-        };
-
-        // owner: add the partial rows of chunk cc from the other CTAs, write o
-        auto finish_rows = [&](int cc) {
-            const int par = cc & 1;
-            if (!warp_wait(&bar[kBarRecv + par], (cc >> 1) & 1, err, 0x301, true)) {
-                ok = false;
-                return;
-            }
-            float z = zheld;
-            for (int sidx = 0; sidx < kNC - 1; ++sidx) {
-                const float *src = recv + (((size_t)par * (4 / kNC) + qtr / kNC) * (kNC - 1) + sidx) *
-                                              (2 * 32 * L::PAY) +
-                                   ((size_t)j * 32 + lane) * L::PAY;
-                for (int e = 0; e < HALF; ++e) held[e] += src[e];
-                z += src[HALF];
-            }
-            const float inv = 1.f / (z + p.eps);
-            if (p.o) {
-                float *dst = p.o + (row0 + (size_t)cc * kC + row) * DH + j * HALF;
-                for (int e = 0; e < HALF; e += 4)
-                    *reinterpret_cast<float4 *>(dst + e) = make_float4(
-                        held[e] * inv, held[e + 1] * inv, held[e + 2] * inv, held[e + 3] * inv);
-            }
-            __syncwarp();
-            // release this chunk's slots in the senders
-            if (lane == 0)
-                for (uint32_t src = 0; src < kNC; ++src)
-                    if (src != rank) mbar_arrive_cluster(&bar[kBarSendFree + 4 * par + qtr], src);
-        };
-
-        for (int c = 0; c < p.nch && ok; ++c) {
-            const int s = c & 1;
-            if (!warp_wait(&bar[kBarFull + s], (c >> 1) & 1, err, 0x302)) { ok = false; break; }
-            const uint8_t *kS = smem + s * L::kStage;
-            const uint8_t *qS = kS + L::kK;
-            // this worker's query row, as bf16 pairs (zero beyond d)
-            uint32_t R[32];
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(qS + sw_off(128, row, ch));
-                R[4 * ch + 0] = v.x;
-                R[4 * ch + 1] = v.y;
-                R[4 * ch + 2] = v.z;
-                R[4 * ch + 3] = v.w;
-            }
-            // K^T into kt (rows a, pitch kKtPitch): this worker writes a in [32 j, 32 j + 32)
-            if (c >= 1 && !warp_wait(&bar[kBarKtFree], (c - 1) & 1, err, 0x30E)) { ok = false; break; }
-            if (j * 32 < DH) {
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(kS + sw_off(128, row, 4 * j + ch));
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int a = 32 * j + 8 * ch + 2 * k;
-                        *reinterpret_cast<uint16_t *>(kt + a * kKtPitch + row * 2) = (uint16_t)(w[k] & 0xFFFFu);
-                        *reinterpret_cast<uint16_t *>(kt + (a + 1) * kKtPitch + row * 2) = (uint16_t)(w[k] >> 16);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bar[kBarKtReady]);
-                mbar_arrive(&bar[kBarEmpty + s]);  // done with this stage's Q and K
-            }
-            if (!warp_wait(&bar[kBarKtReady], c & 1, err, 0x30F)) { ok = false; break; }
-
-            float zpart = 0.f;
-            if (lead) {
-                // S: square, causal mask, row sums; bf16 A operand of the intra product
-                if (!warp_wait(&bar[kBarSReady], c & 1, err, 0x303)) { ok = false; break; }
-                tc_fence_after();
-                for (int h = 0; h < 2; ++h, ++aq) {
-                    const int sl = aq & 1;
-                    uint32_t r[16], pk[16];
-                    // every worker sums all 64 columns of this half (full z per row);
-                    // it converts only its own 32 into the A operand
-                    for (int quarter = 0; quarter < 4; ++quarter) {
-                        const int col0 = 64 * h + 16 * quarter;
-                        tmem_ld16(tmem + lane_base + cS + col0, r);
-                        tmem_ld_wait();
-                        float w16[16];
-                        for (int e = 0; e < 16; ++e) {
-                            const float sv = __uint_as_float(r[e]);
-                            w16[e] = (col0 + e <= row) ? sv * sv : 0.f;
-                            zpart += w16[e];
-                        }
-                        if ((quarter >> 1) == j)
-                            for (int e = 0; e < 8; ++e)
-                                pk[8 * (quarter & 1) + e] = pack_bf16x2(w16[2 * e], w16[2 * e + 1]);
-                    }
-                    if (aq >= 2 && !warp_wait(&bar[kBarAqFree + sl], ((aq >> 1) - 1) & 1, err, 0x304)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    tmem_st16(tmem + lane_base + cAq + 32 * sl + 16 * j, pk);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[kBarAqReady + sl]);
-                }
-                if (!ok) break;
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBarSUsed]);
-                // P = Q G_{c-1}: z_inter = sum_a q_a P_a over this worker's 32 columns
-                if (!warp_wait(&bar[kBarPReady], c & 1, err, 0x305)) { ok = false; break; }
-                tc_fence_after();
-                {
-                    uint32_t r[16];
-#pragma unroll
-                    for (int quarter = 0; quarter < 4; ++quarter) {
-                        tmem_ld16(tmem + lane_base + cS + 16 * quarter, r);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int a = 16 * quarter + e;
-                            const uint32_t w = R[a / 2];
-                            const float qa = __uint_as_float((a & 1) ? (w & 0xFFFF0000u) : (w << 16));
-                            zpart = fmaf(qa, __uint_as_float(r[e]), zpart);
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBarPFree]);
-                // G_c is complete once the G MMA of this chunk is: refresh the mirror
-                if (!warp_wait(&bar[kBarGReady], c & 1, err, 0x306)) { ok = false; break; }
-                tc_fence_after();
-                g_to_mirror();
-            }
-
-            for (int i = 0; i < nt && ok; ++i) {
-                const int g = tb0 + i;
-                // mirror of tile i = H_{c-1} (state after the previous chunk's update)
-                {
-                    const int ms = mr & 1;
-                    if (c >= 1 && !warp_wait(&bar[kBarState + i], (c - 1) & 1, err, 0x307)) { ok = false; break; }
-                    if (mr >= 2 && !warp_wait(&bar[kBarMrFree + ms], ((mr >> 1) - 1) & 1, err, 0x308)) { ok = false; break; }
-                    tc_fence_after();
-                    state_to_mirror(i, ms);
-                    ++mr;
-                }
-                // Phi(Q) for the two 64-row halves of tile g
-                for (int h = 0; h < 2; ++h, ++aq) {
-                    const int sl = aq & 1;
-                    uint32_t out[16];
-                    q_dispatch<DH>(4 * g + 2 * h + j, R, out,
-                                   std::make_integer_sequence<int, 4 * L::NT>{});
-                    if (aq >= 2 && !warp_wait(&bar[kBarAqFree + sl], ((aq >> 1) - 1) & 1, err, 0x309)) { ok = false; break; }
-                    tc_fence_after();
-                    tmem_st16(tmem + lane_base + cAq + 32 * sl + 16 * j, out);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[kBarAqReady + sl]);
-                }
-                if (!ok) break;
-                // Phi(K)^T for packed row (g, row): tokens [64 h + 32 j, +32)
-                {
-                    const uint32_t code = tab[g * 128 + row];
-                    const bool pad = (code >> 16) == 2;
-                    const int a = (code >> 8) & 255, b = code & 255;
-                    const uint8_t *ra = kt + a * kKtPitch, *rb = kt + b * kKtPitch;
-                    for (int h = 0; h < 2; ++h, ++ak) {
-                        const int sl = ak & 1;
-                        uint32_t out[16];
-                        const int t0 = 64 * h + 32 * j;
-#pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
-                            const uint4 x = *reinterpret_cast<const uint4 *>(ra + (t0 + 8 * ch) * 2);
-                            const uint4 y = *reinterpret_cast<const uint4 *>(rb + (t0 + 8 * ch) * 2);
-                            out[4 * ch + 0] = pad ? 0u : hmul2(x.x, y.x);
-                            out[4 * ch + 1] = pad ? 0u : hmul2(x.y, y.y);
-                            out[4 * ch + 2] = pad ? 0u : hmul2(x.z, y.z);
-                            out[4 * ch + 3] = pad ? 0u : hmul2(x.w, y.w);
-                        }
-                        if (ak >= 2 && !warp_wait(&bar[kBarAkFree + sl], ((ak >> 1) - 1) & 1, err, 0x30A)) { ok = false; break; }
-                        tc_fence_after();
-                        tmem_st16(tmem + lane_base + cAk + 32 * sl + 16 * j, out);
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bar[kBarAkReady + sl]);
-                    }
-                }
-            }
-            if (!ok) break;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kBarKtFree]);
-
-            // epilogue: this CTA's partial O rows -> owner
-            if (!warp_wait(&bar[kBarOReady], c & 1, err, 0x30B)) { ok = false; break; }
-            tc_fence_after();
-            float part[HALF];
-            if (nt == 0 && !lead) {
-                for (int e = 0; e < HALF; ++e) part[e] = 0.f;
-            } else {
-                uint32_t r[16];
-                for (int c0 = 0; c0 < HALF; c0 += 16) {
-                    tmem_ld16(tmem + lane_base + cO + j * HALF + c0, r);
-                    tmem_ld_wait();
-                    for (int e = 0; e < 16; ++e) part[c0 + e] = __uint_as_float(r[e]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kBarOFree]);
-            if (own) {
-                if (held_c >= 0) finish_rows(held_c);
-                if (!ok) break;
-                for (int e = 0; e < HALF; ++e) held[e] = part[e];
-                zheld = lead ? zpart : 0.f;
-                held_c = c;
-            } else {
-                // the owner has released this parity's slot (chunk c - 2 consumed)
-                if (c >= 2 && !warp_wait(&bar[kBarSendFree + 4 * (c & 1) + qtr], ((c >> 1) - 1) & 1,
-                                         err, 0x30C, true)) {
-                    ok = false;
-                    break;
-                }
-                const int par = c & 1;
-                const uint32_t sidx = (rank + kNC - owner - 1) % kNC;
-                float *slot = recv + (((size_t)par * (4 / kNC) + qtr / kNC) * (kNC - 1) + sidx) *
-                                         (2 * 32 * L::PAY) +
-                              ((size_t)j * 32 + lane) * L::PAY;
-                const uint32_t a0 = smem_u32(slot);
-                for (int e = 0; e < HALF; e += 4)
-                    st_cluster_v4(a0 + e * 4, owner, part[e], part[e + 1], part[e + 2], part[e + 3]);
-                st_cluster_v4(a0 + HALF * 4, owner, lead ? zpart : 0.f, 0.f, 0.f, 0.f);
-                mbar_arrive_cluster(&bar[kBarRecv + par], owner);
-            }
-        }
-        if (ok && own && held_c >= 0) finish_rows(held_c);
-
-        // final state -> H_out (packed, with sqrt 2), G -> s_out
-        if (ok && (p.H_out || p.s_out)) {
-            if (!warp_wait(&bar[kBarFinal], 0, err, 0x30D)) ok = false;
-            tc_fence_after();
-            if (ok && p.H_out) {
-                for (int i = 0; i < nt; ++i) {
-                    const uint32_t code = tab[(tb0 + i) * 128 + row];
-                    const int a = (code >> 8) & 255, b = code & 255;
-                    const bool pad = (code >> 16) == 2;
-                    const float w = (a == b) ? 1.f : 1.41421356237309515f;
-                    uint32_t r[16];
-                    for (int c0 = 0; c0 < HALF; c0 += 16) {
-                        tmem_ld16(tmem + lane_base + i * DH + j * HALF + c0, r);
-                        tmem_ld_wait();
-                        if (!pad) {
-                            float *dst = p.H_out + ((size_t)bh * D + canon_index(DH, a, b)) * DH +
-                                         j * HALF + c0;
-                            for (int e = 0; e < 16; e += 4)
-                                *reinterpret_cast<float4 *>(dst + e) = make_float4(
-                                    __uint_as_float(r[e]) * w, __uint_as_float(r[e + 1]) * w,
-                                    __uint_as_float(r[e + 2]) * w, __uint_as_float(r[e + 3]) * w);
-                        }
-                    }
-                }
-            }
-            if (ok && p.s_out && lead && qtr < 2) {
-                uint32_t r[16];
-                for (int c0 = 0; c0 < 32; c0 += 16) {
-                    tmem_ld16(tmem + lane_base + cG + j * 32 + c0, r);
-                    tmem_ld_wait();
-                    for (int e = 0; e < 16; ++e) {
-                        const int b = j * 32 + c0 + e;
-                        if (row < DH && b >= row && b < DH)
-                            p.s_out[(size_t)bh * D + canon_index(DH, row, b)] =
-                                __uint_as_float(r[e]) * (b == row ? 1.f : 1.41421356237309515f);
-                    }
-                }
-            }
-        }
-    }
-
-    // ---- teardown ------------------------------------------------------
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) {
-        // wait (bounded) for the last MMAs before releasing tensor memory
-        if (lane == 0) mbar_wait(&bar[kBarFinal], 0, err, 0x401, 1u << 22);
-        __syncwarp();
-        tmem_dealloc(tmem, 512);
+    const uint32_t tmem = *tmem_slot;
+    const long row0 = (long)head * p.nch * kTile;  // first token row of this head
+
+    if (warp == 5) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            prefetch_tensormap(&mk);
+            prefetch_tensormap(&mv);
+            for (int c = 0; c < p.nch; ++c) {
+                const int s = c & 1, n = c >> 1;
+                if (n > 0) mbar_wait(&bar[kSbKFree + s], (n - 1) & 1, err, 0x401);
+                mbar_arrive_expect_tx(&bar[kSbKFull + s], kTileBytes);
+                tma_load_2d(sm + L::K0 + s * kTileBytes, &mk, 0, (int)(row0 + c * kTile),
+                            &bar[kSbKFull + s]);
+                if (n > 0) mbar_wait(&bar[kSbVFree + s], (n - 1) & 1, err, 0x402);
+                mbar_arrive_expect_tx(&bar[kSbVFull + s], kTileBytes);
+                tma_load_2d(sm + L::V0 + s * kTileBytes, &mv, 0, (int)(row0 + c * kTile),
+                            &bar[kSbVFull + s]);
+            }
+            // no copy may still be in flight when the CTA exits
+            for (int c = p.nch - 2 < 0 ? 0 : p.nch - 2; c < p.nch; ++c) {
+                mbar_wait(&bar[kSbKFull + (c & 1)], (c >> 1) & 1, err, 0x403);
+                mbar_wait(&bar[kSbVFull + (c & 1)], (c >> 1) & 1, err, 0x404);
+            }
+        }
+    } else if (warp == 4) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, kAccCols, 0, 1);
+            const uint32_t ones = smem_u32(sm + L::ONES);
+            for (int c = 0; c < p.nch; ++c) {
+                const int s = c & 1;
+                mbar_wait(&bar[kSbAFull + s], (c >> 1) & 1, err, 0x410);
+                // the state at an interval end must be read before it moves on
+                if (c > 0 && c % p.cpi == 0)
+                    mbar_wait(&bar[kSbSnap], (c / p.cpi - 1) & 1, err, 0x411);
+                mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412);
+                tc_fence_after();
+                const uint32_t v = smem_u32(sm + L::V0 + s * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    mma_ts(tmem + kStAcc, tmem + kStA + 64 * s + 8 * kk,
+                           vones_desc(v, ones, 16 * kk), idesc, 1);
+                mma_commit(&bar[kSbVFree + s]);
+                mma_commit(&bar[kSbDone + s]);
+            }
+        }
+    } else {
+        // ---------------- workers: one thread per feature row ----------------
+        const int f = threadIdx.x;  // tensor-memory lane = row of this state tile
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int slice = 2 * tile + (f >> 6);
+        const bool valid = slice < S::NS;
+        int ra = 0, rb = 0;
+        if (valid) {
+            int A, B;
+            slice_blocks(slice, S::NB, A, B);
+            ra = 8 * A + ((f & 63) >> 3);
+            rb = 8 * B + (f & 7);
+        }
+        uint8_t *kt = sm + L::KT;
+
+        // all-ones atom of the [V | 1] operand
+        {
+            uint4 *o4 = reinterpret_cast<uint4 *>(sm + L::ONES);
+            for (int i = f; i < kTileBytes / 16; i += kWorkers)
+                o4[i] = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
+            fence_proxy_async_smem();
+        }
+
+        // initial state: H_in in the internal scaling (no sqrt 2), or zero
+        float init[DH + 1];
+        {
+            const bool have = valid && p.H_in != nullptr;
+            const int ci = valid ? canon_index(ra, rb, DH) : 0;
+            const float w = (ra != rb) ? 0.70710678118654752f : 1.f;
+            const size_t hb = ((size_t)head * (DH * (DH + 1) / 2) + ci);
+#pragma unroll
+            for (int n = 0; n < DH; ++n) init[n] = have ? p.H_in[hb * DH + n] * w : 0.f;
+            init[DH] = have ? p.s_in[hb] * w : 0.f;
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < kAccCols / 16; ++j) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int col = 16 * j + e;
+                    const float x = col < DH ? init[col] : (col >= kSCol ? init[DH] : 0.f);
+                    r[e] = __float_as_uint(x);
+                }
+                tmem_st16(tmem + lane_base + kStAcc + 16 * j, r);
+            }
+            tmem_st_wait();
+        }
+        // snapshot writer: rows n < DH take column n, rows DH.. take s
+        auto write_snapshot = [&](int g, const float (&x)[DH + 1]) {
+            if (!valid || p.snap == nullptr) return;
+            uint8_t *dst = p.snap +
+                           (((size_t)head * p.nint + g) * S::NS + slice) * S::SLICE_BYTES;
+            const int fl = f & 63;
+#pragma unroll
+            for (int n = 0; n < S::NSNAP; ++n) {
+                const float val = n < DH ? x[n] : x[DH];
+                const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+                const uint32_t nb = __shfl_down_sync(0xFFFFFFFFu, h, 1);
+                if ((fl & 1) == 0)
+                    *reinterpret_cast<uint32_t *>(dst + n * 128 + (((fl >> 3) ^ (n & 7)) << 4) +
+                                                  (fl & 7) * 2) = h | (nb << 16);
+            }
+        };
+        if (p.H_in) write_snapshot(0, init);
+        // accumulator columns 0..DH-1 and the s column
+        auto read_acc = [&](float (&x)[DH + 1]) {
+            const uint32_t acc = tmem + lane_base + kStAcc;
+#pragma unroll
+            for (int j = 0; j < DH / 16; ++j) {
+                float y[16];
+                tmem_ld16_f(acc + 16 * j, y);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) x[16 * j + e] = y[e];
+            }
+            float y[16];
+            tmem_ld16_f(acc + kSCol, y);
+            x[DH] = y[0];
+        };
+
+        for (int c = 0; c < p.nch; ++c) {
+            const int s = c & 1;
+            // transpose the K tile: thread = token
+            warp_wait(&bar[kSbKFull + s], (c >> 1) & 1, err, 0x420);
+            {
+                const uint8_t *kb = sm + L::K0 + s * kTileBytes;
+                const int t = f;
+#pragma unroll
+                for (int j = 0; j < DH / 8; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(kb + sw128_chunk(t, j));
+                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        *reinterpret_cast<uint16_t *>(kt + (8 * j + 2 * e) * kKtPitch + 2 * t) =
+                            (uint16_t)(w4[e] & 0xFFFFu);
+                        *reinterpret_cast<uint16_t *>(kt + (8 * j + 2 * e + 1) * kKtPitch + 2 * t) =
+                            (uint16_t)(w4[e] >> 16);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kSbKFree + s]);
+            worker_sync();  // K^T complete
+            // Phi(K)^T row of feature (ra, rb): 128 tokens, two per 32-bit column
+            uint32_t a_row[64];
+            {
+                const uint8_t *pa = kt + ra * kKtPitch, *pb = kt + rb * kKtPitch;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(pa + 16 * j);
+                    const uint4 y = *reinterpret_cast<const uint4 *>(pb + 16 * j);
+                    a_row[4 * j + 0] = valid ? hmul2(x.x, y.x) : 0u;
+                    a_row[4 * j + 1] = valid ? hmul2(x.y, y.y) : 0u;
+                    a_row[4 * j + 2] = valid ? hmul2(x.z, y.z) : 0u;
+                    a_row[4 * j + 3] = valid ? hmul2(x.w, y.w) : 0u;
+                }
+            }
+            worker_sync();  // K^T free for the next chunk
+            // A slot s was last read by chunk c - 2
+            if (c >= 2) warp_wait(&bar[kSbDone + s], ((c >> 1) - 1) & 1, err, 0x421);
+            tc_fence_after();
+            {
+                uint32_t r[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) r[e] = a_row[16 * j + e];
+                    tmem_st16(tmem + lane_base + kStA + 64 * s + 16 * j, r);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kSbAFull + s]);
+            // chunk c opens interval g: the state after chunk c - 1 is snapshot g
+            // (A(c) is already published, so the issuer waits only for this read)
+            if (c > 0 && c % p.cpi == 0) {
+                const int sp = (c - 1) & 1;
+                warp_wait(&bar[kSbDone + sp], ((c - 1) >> 1) & 1, err, 0x422);
+                tc_fence_after();
+                float x[DH + 1];
+                read_acc(x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kSbSnap]);
+                write_snapshot(c / p.cpi, x);
+            }
+        }
+        // final state, converted to the canonical layout
+        warp_wait(&bar[kSbDone + ((p.nch - 1) & 1)], ((p.nch - 1) >> 1) & 1, err, 0x423);
+        tc_fence_after();
+        if (p.H_out) {
+            float fin[DH + 1];
+            read_acc(fin);
+            if (valid && ra <= rb) {
+                const int ci = canon_index(ra, rb, DH);
+                const float w = (ra != rb) ? 1.41421356237309505f : 1.f;
+                const size_t hb = (size_t)head * (DH * (DH + 1) / 2) + ci;
+                float4 *dst = reinterpret_cast<float4 *>(p.H_out + hb * DH);
+#pragma unroll
+                for (int n = 0; n < DH; n += 4)
+                    dst[n / 4] = make_float4(fin[n] * w, fin[n + 1] * w, fin[n + 2] * w,
+                                             fin[n + 3] * w);
+                p.s_out[hb] = fin[DH] * w;
+            }
+        }
     }
-    cluster_sync();  // no CTA leaves while another may still write its shared memory
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
 }
 
-// ------------------------------------------------------------------ host ---
+// ---------------------------------------------------------------------------
+// Readout kernel
+// ---------------------------------------------------------------------------
+
+constexpr int kRP = 4;  // snapshot slices in flight
+constexpr int kRQ = 3;  // A-operand slots in tensor memory
+
+struct ReadParams {
+    int nch;     // query tiles (= chunks) per head
+    int cpi;     // chunks per snapshot interval
+    int nint;    // snapshot intervals per head
+    int has_in;  // an initial state was given: snapshot 0 exists
+    const uint8_t *snap;
+    float *o;
+    float eps;
+    unsigned int *err;
+};
+
+enum ReadBar {
+    kRbQFull = 0,
+    kRbKFull = 1,
+    kRbKFree = 2,
+    kRbVFull = 3,
+    kRbVFree = 4,
+    kRbSFull = 5,
+    kRbSFree = 6,  // 4 warp arrivals
+    kRbODone = 7,
+    kRbPFull = 8,
+    kRbPFree = kRbPFull + kRP,
+    kRbAqFull = kRbPFree + kRP,  // 4 warp arrivals
+    kRbAqFree = kRbAqFull + kRQ,
+    kRbCount = kRbAqFree + kRQ
+};
+
+template <int DH>
+struct ReadSmem {
+    static constexpr int Q = 0;
+    static constexpr int K = kTileBytes;
+    static constexpr int V = 2 * kTileBytes;
+    static constexpr int ONES = 3 * kTileBytes;
+    static constexpr int P = 4 * kTileBytes;  // kRP snapshot slices
+    static constexpr int BAR = P + kRP * Shape<DH>::SLICE_BYTES;
+    static constexpr int SLOT = BAR + kRbCount * 8;
+    static constexpr int BYTES = SLOT + 16 + 1024;
+};
+
+// Tensor-memory columns of the readout kernel (256 allocated).
+constexpr uint32_t kRdO = 0, kRdS = 96, kRdAq = 160;
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 2)
+    readout_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                   const __grid_constant__ CUtensorMap mv, ReadParams p) {
+    using S = Shape<DH>;
+    using L = ReadSmem<DH>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m = blockIdx.x, head = blockIdx.y;  // query tile, (batch, head)
+    unsigned int *err = p.err;
+
+    const int g = m / p.cpi;             // snapshot interval of this query tile
+    const int kt0 = g * p.cpi;           // first key tile of the interval
+    const int n_half = 2 * (m - kt0 + 1);  // intra items: 64-key halves
+    const int n_inter = (g > 0 || p.has_in) ? S::NS : 0;
+    const int n_items = n_half + n_inter;
+    const long row0 = (long)head * p.nch * kTile;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kRbCount; ++i) {
+            const bool four = i == kRbSFree || (i >= kRbAqFull && i < kRbAqFull + kRQ);
+            mbar_init(&bar[i], four ? 4 : 1);
+        }
+        fence_barrier_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint8_t *snap =
+        p.snap + ((size_t)head * p.nint + g) * S::NS * (size_t)S::SLICE_BYTES;
+
+    if (warp == 5) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            prefetch_tensormap(&mq);
+            prefetch_tensormap(&mk);
+            prefetch_tensormap(&mv);
+            auto load_p = [&](int s) {
+                const int slot = s % kRP;
+                if (s >= kRP) mbar_wait(&bar[kRbPFree + slot], ((s / kRP) - 1) & 1, err, 0x501);
+                mbar_arrive_expect_tx(&bar[kRbPFull + slot], S::SLICE_BYTES);
+                bulk_load(sm + L::P + slot * S::SLICE_BYTES, snap + (size_t)s * S::SLICE_BYTES,
+                          S::SLICE_BYTES, &bar[kRbPFull + slot]);
+            };
+            auto load_kv = [&](int u) {
+                const int y = (int)(row0 + (long)(kt0 + u) * kTile);
+                if (u > 0) mbar_wait(&bar[kRbKFree], (u - 1) & 1, err, 0x502);
+                mbar_arrive_expect_tx(&bar[kRbKFull], kTileBytes);
+                tma_load_2d(sm + L::K, &mk, 0, y, &bar[kRbKFull]);
+                if (u > 0) mbar_wait(&bar[kRbVFree], (u - 1) & 1, err, 0x503);
+                mbar_arrive_expect_tx(&bar[kRbVFull], kTileBytes);
+                tma_load_2d(sm + L::V, &mv, 0, y, &bar[kRbVFull]);
+            };
+            mbar_arrive_expect_tx(&bar[kRbQFull], kTileBytes);
+            tma_load_2d(sm + L::Q, &mq, 0, (int)(row0 + (long)m * kTile), &bar[kRbQFull]);
+            load_kv(0);
+            const int first_p = n_inter < kRP ? n_inter : kRP;
+            for (int s = 0; s < first_p; ++s) load_p(s);
+            for (int u = 1; u < n_half / 2; ++u) load_kv(u);
+            for (int s = first_p; s < n_inter; ++s) load_p(s);
+            // no copy may still be in flight when the CTA exits
+            mbar_wait(&bar[kRbQFull], 0, err, 0x504);
+            const int nu = n_half / 2;
+            mbar_wait(&bar[kRbKFull], (nu - 1) & 1, err, 0x505);
+            mbar_wait(&bar[kRbVFull], (nu - 1) & 1, err, 0x506);
+            for (int s = n_inter - kRP < 0 ? 0 : n_inter - kRP; s < n_inter; ++s)
+                mbar_wait(&bar[kRbPFull + s % kRP], (s / kRP) & 1, err, 0x507);
+        }
+    } else if (warp == 4) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t i_s = idesc_bf16(128, 64, 0, 0);
+            const uint32_t i_av = idesc_bf16(128, kAccCols, 0, 1);
+            const uint32_t i_p = idesc_bf16(128, S::NSNAP, 0, 0);
+            const uint32_t q_a = smem_u32(sm + L::Q), k_a = smem_u32(sm + L::K);
+            const uint32_t v_a = smem_u32(sm + L::V), ones = smem_u32(sm + L::ONES);
+            auto issue_s = [&](int j) {  // S = Q K^T for 64-key half j
+                const int u = j >> 1, h = j & 1;
+                if (h == 0) mbar_wait(&bar[kRbKFull], u & 1, err, 0x510);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk)
+                    mma_ss(tmem + kRdS, kmaj_desc(q_a, kk), kmaj_desc(k_a + h * 64 * 128, kk), i_s,
+                           kk > 0);
+                mma_commit(&bar[kRbSFull]);
+                if (h == 1) mma_commit(&bar[kRbKFree]);
+            };
+            mbar_wait(&bar[kRbQFull], 0, err, 0x511);
+            issue_s(0);
+            for (int it = 0; it < n_items; ++it) {
+                const int slot = it % kRQ;
+                if (it < n_half) {
+                    const int j = it, h = j & 1;
+                    if (j + 1 < n_half) {
+                        mbar_wait(&bar[kRbSFree], j & 1, err, 0x512);
+                        issue_s(j + 1);
+                    }
+                    mbar_wait(&bar[kRbAqFull + slot], (it / kRQ) & 1, err, 0x513);
+                    if (h == 0) mbar_wait(&bar[kRbVFull], (j >> 1) & 1, err, 0x514);
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + kRdO, tmem + kRdAq + 32 * slot + 8 * kk,
+                               vones_desc(v_a, ones, 64 * h + 16 * kk), i_av, 1);
+                    mma_commit(&bar[kRbAqFree + slot]);
+                    if (h == 1) mma_commit(&bar[kRbVFree]);
+                } else {
+                    const int s = it - n_half, ps = s % kRP;
+                    mbar_wait(&bar[kRbAqFull + slot], (it / kRQ) & 1, err, 0x515);
+                    mbar_wait(&bar[kRbPFull + ps], (s / kRP) & 1, err, 0x516);
+                    tc_fence_after();
+                    const uint32_t pa = smem_u32(sm + L::P + ps * S::SLICE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + kRdO, tmem + kRdAq + 32 * slot + 8 * kk, kmaj_desc(pa, kk),
+                               i_p, 1);
+                    mma_commit(&bar[kRbAqFree + slot]);
+                    mma_commit(&bar[kRbPFree + ps]);
+                }
+            }
+            mma_commit(&bar[kRbODone]);
+        }
+    } else {
+        // ---------------- workers: one thread per query row ----------------
+        const int i = threadIdx.x;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        {
+            uint32_t z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) z[e] = 0u;
+#pragma unroll
+            for (int j = 0; j < kAccCols / 16; ++j) tmem_st16(tmem + lane_base + kRdO + 16 * j, z);
+            tmem_st_wait();
+            uint4 *o4 = reinterpret_cast<uint4 *>(sm + L::ONES);
+            for (int x = i; x < kTileBytes / 16; x += kWorkers)
+                o4[x] = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
+            fence_proxy_async_smem();
+        }
+        warp_wait(&bar[kRbQFull], 0, err, 0x520);
+        for (int it = 0; it < n_items; ++it) {
+            const int slot = it % kRQ;
+            uint32_t pk[32];
+            if (it < n_half) {
+                // intra: squared scores of 64 keys, causal mask on the diagonal tile
+                const int j = it, h = j & 1, u = j >> 1;
+                const bool diag = kt0 + u == m;
+                warp_wait(&bar[kRbSFull], j & 1, err, 0x521);
+                tc_fence_after();
+                float sv[64];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem + lane_base + kRdS + 16 * q4, r);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[16 * q4 + e] = __uint_as_float(r[e]);
+                }
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kRbSFree]);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int k0 = 64 * h + 2 * e;
+                    const float a0 = (diag && k0 > i) ? 0.f : sv[2 * e] * sv[2 * e];
+                    const float a1 = (diag && k0 + 1 > i) ? 0.f : sv[2 * e + 1] * sv[2 * e + 1];
+                    pk[e] = pack_bf16x2(a0, a1);
+                }
+            } else {
+                // inter: Phi(Q) for slice s, block pair (A, B); q[8A..8A+7] and
+                // q[8B..8B+7] are 16-byte chunks A and B of this row of the Q tile
+                int A, B;
+                slice_blocks(it - n_half, S::NB, A, B);
+                const uint32_t wgt = A < B ? 0x40004000u : 0x3F803F80u;  // 2 or 1
+                const uint4 xa = *reinterpret_cast<const uint4 *>(sm + L::Q + sw128_chunk(i, A));
+                const uint4 xb = *reinterpret_cast<const uint4 *>(sm + L::Q + sw128_chunk(i, B));
+                const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w};
+                const uint32_t wb[4] = {xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                for (int a = 0; a < 8; ++a) {
+                    const uint32_t qa =
+                        hmul2((a & 1) ? bcast_hi(wa[a >> 1]) : bcast_lo(wa[a >> 1]), wgt);
+#pragma unroll
+                    for (int bb = 0; bb < 4; ++bb) pk[4 * a + bb] = hmul2(qa, wb[bb]);
+                }
+            }
+            if (it >= kRQ) warp_wait(&bar[kRbAqFree + slot], ((it / kRQ) - 1) & 1, err, 0x522);
+            tc_fence_after();
+            {
+                uint32_t r[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = pk[e];
+                tmem_st16(tmem + lane_base + kRdAq + 32 * slot, r);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = pk[16 + e];
+                tmem_st16(tmem + lane_base + kRdAq + 32 * slot + 16, r);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kRbAqFull + slot]);
+        }
+        // epilogue: o = numerator / (denominator + eps)
+        warp_wait(&bar[kRbODone], 0, err, 0x523);
+        tc_fence_after();
+        float den;
+        {
+            float x[16];
+            tmem_ld16_f(tmem + lane_base + kRdO + kSCol, x);
+            den = x[0];
+            if (DH < kSCol) {
+                tmem_ld16_f(tmem + lane_base + kRdO + DH, x);
+                den += x[0];
+            }
+        }
+        const float inv = 1.f / (den + p.eps);
+        float4 *dst =
+            reinterpret_cast<float4 *>(p.o + ((size_t)head * p.nch * kTile + (size_t)m * kTile + i) * DH);
+#pragma unroll
+        for (int j = 0; j < DH / 16; ++j) {
+            float x[16];
+            tmem_ld16_f(tmem + lane_base + kRdO + 16 * j, x);
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                dst[4 * j + e / 4] = make_float4(x[e] * inv, x[e + 1] * inv, x[e + 2] * inv,
+                                                 x[e + 3] * inv);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -833,87 +742,91 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *base, int d, long rows, int box_x,
-              CUtensorMapSwizzle sw) {
+// [rows, d] bf16 rows, 128 x 64 boxes with the 128-byte swizzle; for d = 32
+// the box reaches past the row and the extra columns are zero-filled.
+bool make_map(CUtensorMap *m, const void *base, int d, long rows) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)kC};
+    cuuint32_t box[2] = {64, (cuuint32_t)kTile};
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
+// Chunks per snapshot interval: longer intervals mean fewer snapshot bytes
+// and more quadratic intra work per query tile.
+int chunks_per_interval(int d, int nch) {
+    int c = d == 64 ? 4 : 1;
+    while (c > 1 && nch % c) c >>= 1;
+    return c;
+}
+
 template <int DH>
-cudaError_t launch_tc(const PrefillArgs &a, cudaStream_t stream) {
-    using L = Layout<DH>;
+size_t snapshot_bytes(long nheads, int nch) {
+    const int nint = nch / chunks_per_interval(DH, nch);
+    return (size_t)nheads * nint * Shape<DH>::NS * Shape<DH>::SLICE_BYTES;
+}
+
+template <int DH>
+cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
+    using S = Shape<DH>;
+    const int nheads = a.B * a.H, nch = a.T / kTile;
+    const int cpi = chunks_per_interval(DH, nch), nint = nch / cpi;
+    const long rows = (long)nheads * a.T;
+    const bool want_o = a.o != nullptr;
+    uint8_t *snap = want_o ? static_cast<uint8_t *>(a.ws) : nullptr;
+    if (want_o && a.ws_bytes < snapshot_bytes<DH>(nheads, nch)) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
-    const long rows = (long)a.B * a.H * a.T;
-    if (!make_map(&mq, a.q, DH, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mk, a.k, DH, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mv, a.v, DH, rows, DH,
-                  DH == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map(&mq, a.q, DH, rows) || !make_map(&mk, a.k, DH, rows) ||
+        !make_map(&mv, a.v, DH, rows))
         return cudaErrorInvalidValue;
-    TcParams p{};
-    p.T = a.T;
-    p.nch = a.T / kC;
-    p.nheads = a.B * a.H;
-    p.eps = a.eps;
-    // rank 0 also does the intra-chunk part and G: give it fewer tiles
-    const int nt = L::NT;
-    const int t0 = DH == 64 ? 2 : 1;
-    p.tile_begin[0] = 0;
-    p.tile_begin[1] = t0;
+
+    StateParams sp{nch, cpi, nint, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
     {
-        const int rest = nt - t0, base = rest / (kNC - 1), rem = rest % (kNC - 1);
-        for (int r = 1; r < kNC; ++r)
-            p.tile_begin[r + 1] = p.tile_begin[r] + base + (r <= rem ? 1 : 0);
+        auto kern = state_kernel<DH>;
+        const int bytes = StateSmem<DH>::BYTES;
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3(S::NT, nheads), kThreads, bytes, stream>>>(mk, mv, sp);
+        e = after_launch();
+        if (e != cudaSuccess) return e;
     }
-    p.H_in = a.H_in;
-    p.s_in = a.s_in;
-    p.o = a.o;
-    p.H_out = a.H_out;
-    p.s_out = a.s_out;
-    p.err = a.err;
-    auto kern = prefill_tc_kernel<DH>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::kBytes);
+    if (!want_o) return cudaSuccess;
+    ReadParams rp{nch, cpi, nint, a.H_in != nullptr ? 1 : 0, snap, a.o, a.eps, a.err};
+    auto kern = readout_kernel<DH>;
+    const int bytes = ReadSmem<DH>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(kNC, a.B * a.H, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = L::kBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kNC;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
-    if (e != cudaSuccess) return e;
+    kern<<<dim3(nch, nheads), kThreads, bytes, stream>>>(mq, mk, mv, rp);
     return after_launch();
 }
 
 }  // namespace
 
 bool prefill_tc_supported(const PrefillArgs &a) {
-    return a.dtype == 1 && (a.d == 64 || a.d == 32) && a.T % kC == 0 &&
+    return a.dtype == 1 && (a.d == 64 || a.d == 32) && a.T % kTile == 0 &&
+           (long)a.B * a.H * a.T < (1L << 31) && a.B * a.H <= 65535 &&
            (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(a.k) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(a.v) & 15) == 0;
+           (reinterpret_cast<uintptr_t>(a.v) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(a.ws) & 15) == 0;
 }
 
-size_t prefill_tc_workspace_bytes(int, int, int, int, int) { return 0; }
+size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int) {
+    if (T % kTile) return 0;
+    if (d == 32) return snapshot_bytes<32>((long)B * H, T / kTile);
+    if (d == 64) return snapshot_bytes<64>((long)B * H, T / kTile);
+    return 0;
+}
 
 cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
-    return a.d == 64 ? launch_tc<64>(a, stream) : launch_tc<32>(a, stream);
+    return a.d == 64 ? launch<64>(a, stream) : launch<32>(a, stream);
 }
 
 }  // namespace kata
