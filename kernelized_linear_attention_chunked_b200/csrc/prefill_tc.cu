@@ -57,7 +57,6 @@ constexpr int kTile = 128;         // tokens per chunk / query tile; rows per st
 constexpr int kTileBytes = 16384;  // one 128 x 64 bf16 tile, 128-byte swizzle
 constexpr int kAccCols = 80;       // accumulator columns: H (<= 64) | s x 16
 constexpr int kSCol = 64;          // first accumulator column holding s
-constexpr int kKtPitch = 272;      // bytes per row of the transposed K tile (256 + 16)
 constexpr int kWorkers = 128;      // 4 warps: one thread per tensor-memory lane
 constexpr int kThreads = 192;      // + MMA issuer warp + TMA producer warp
 constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
@@ -125,9 +124,11 @@ __device__ __forceinline__ void tmem_ld16_f(uint32_t taddr, float (&f)[16]) {
 
 // MN-major [V | 1] operand for 16 tokens starting at row `row0` of the V tile:
 // the V tile (64 bf16 per row, zero-filled past d) is the first 64-column
-// atom, the all-ones tile the second, `ones - v` bytes further on.
+// atom; the second atom is a 16-row all-ones block, reached through the
+// leading byte offset from this K-step's start (every row of it is the same).
 __device__ __forceinline__ uint64_t vones_desc(uint32_t v, uint32_t ones, int row0) {
-    return smem_desc(v + row0 * 128, ones - v, 1024, kSwizzle128);
+    const uint32_t start = v + row0 * 128;
+    return smem_desc(start, ones - start, 1024, kSwizzle128);
 }
 
 // K-major operand: 128-byte rows, 16 K-elements at byte offset 32 * kk.
@@ -145,42 +146,54 @@ struct StateParams {
     int nint;       // snapshot intervals per head
     const float *H_in, *s_in;
     float *H_out, *s_out;
-    uint8_t *snap;  // [heads][nint][NS][NSNAP][128 B]
+    uint8_t *snap;  // [heads][nint][NS][NSNAP][128 B], or null: no snapshots
     unsigned int *err;
 };
 
 enum StateBar {
-    kSbKFull = 0,     // 2: K tile landed
-    kSbKFree = 2,     // 2: the workers transposed it (4 warp arrivals)
-    kSbVFull = 4,     // 2: V tile landed
-    kSbVFree = 6,     // 2: the chunk's MMAs finished reading it
-    kSbAFull = 8,     // 2: Phi(K)^T tile written to tensor memory (4 warp arrivals)
-    kSbDone = 10,     // 2: the MMAs of the chunk that used this A slot completed
-    kSbSnap = 12,     // the workers read the accumulator at an interval end (4 warp arrivals)
-    kSbCount = 13
+    kSbKFull = 0,    // 4: K tile landed
+    kSbKFree = 4,    // 4: the workers transposed it (4 warp arrivals)
+    kSbVFull = 8,    // 2: V tile landed
+    kSbVFree = 10,   // 2: the chunk's MMAs finished reading it (one commit per issuer)
+    kSbAFull = 12,   // NA: Phi(K)^T tile written to tensor memory (4 warp arrivals)
+    kSbDone = 14,    // NA: the MMAs of the chunk that used this A slot completed
+    kSbSnap = 16,    // the workers read the accumulators at an interval end
+    kSbCount = 17
 };
 
-template <int DH>
-struct StateSmem {
-    static constexpr int K0 = 0;                      // 2 x K tile
-    static constexpr int V0 = 2 * kTileBytes;         // 2 x V tile
-    static constexpr int ONES = 4 * kTileBytes;       // all-ones atom
-    static constexpr int KT = 5 * kTileBytes;         // K^T, DH rows of kKtPitch bytes
-    static constexpr int BAR = KT + DH * kKtPitch;    // barriers
-    static constexpr int SLOT = BAR + kSbCount * 8;   // tensor-memory base address
-    static constexpr int BYTES = SLOT + 16 + 1024;    // + alignment slack
+// Transposed K tile: row a holds k[t][a] for the 128 tokens of the chunk as
+// 16 chunks of 16 bytes; chunk j of row a sits at j ^ kt_swz(a), which keeps
+// both the 8x8 block transpose writes and the per-feature row reads free of
+// shared-memory bank conflicts.
+__device__ __forceinline__ uint32_t kt_offset(int row, int chunk) {
+    return (uint32_t)(row * 256 + ((chunk ^ ((row + (row >> 3)) & 7)) << 4));
+}
+
+template <int DH, int NI, int NA>
+struct StateCfg {
+    static constexpr int KR = DH == 64 ? 2 : 3;  // K tiles in flight
+    static constexpr int K0 = 0;
+    static constexpr int V0 = KR * kTileBytes;    // 2 x V tile
+    static constexpr int ONES = V0 + 2 * kTileBytes;
+    static constexpr int KT = ONES + 2048;
+    static constexpr int STAGE = KT + DH * 256;   // snapshot staging: 2 slices
+    static constexpr int BAR = STAGE + 2 * Shape<DH>::SLICE_BYTES;
+    static constexpr int SLOT = BAR + kSbCount * 8;
+    static constexpr int BYTES = SLOT + 16 + 1024;
+    static constexpr int THREADS = 32 * (5 + NI);  // workers, NI issuers, TMA
+    // NI accumulators of 80 columns at a 96-column pitch, then NA Phi(K)^T slots
+    static constexpr uint32_t A_COL = 96u * NI;
+    static constexpr uint32_t TMEM_COLS = A_COL + 64u * NA <= 256 ? 256 : 512;
+    __host__ __device__ static constexpr uint32_t acc_col(int i) { return 96u * i; }
 };
 
-// Tensor-memory columns of the state kernel (256 allocated): the fp32
-// accumulator and two Phi(K)^T slots (128 tokens as bf16 pairs each).
-constexpr uint32_t kStAcc = 0, kStA = 128;
-
-template <int DH>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int DH, int NI, int NA>
+__global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
+                                  StateCfg<DH, NI, NA>::TMEM_COLS == 256 ? 2 : 1)
     state_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
                  StateParams p) {
     using S = Shape<DH>;
-    using L = StateSmem<DH>;
+    using L = StateCfg<DH, NI, NA>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -189,21 +202,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = blockIdx.x, head = blockIdx.y;
     unsigned int *err = p.err;
+    constexpr int kTmaWarp = 4 + NI;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < L::KR; ++i) {
             mbar_init(&bar[kSbKFull + i], 1);
             mbar_init(&bar[kSbKFree + i], 4);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bar[kSbVFull + i], 1);
-            mbar_init(&bar[kSbVFree + i], 1);
+            mbar_init(&bar[kSbVFree + i], NI);
+        }
+        for (int i = 0; i < NA; ++i) {
             mbar_init(&bar[kSbAFull + i], 4);
-            mbar_init(&bar[kSbDone + i], 1);
+            mbar_init(&bar[kSbDone + i], NI);
         }
         mbar_init(&bar[kSbSnap], 4);
         fence_barrier_init();
     }
     if (warp == 4) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -212,48 +230,71 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const long row0 = (long)head * p.nch * kTile;  // first token row of this head
 
-    if (warp == 5) {
+    if (warp == kTmaWarp) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&mk);
             prefetch_tensormap(&mv);
-            for (int c = 0; c < p.nch; ++c) {
-                const int s = c & 1, n = c >> 1;
-                if (n > 0) mbar_wait(&bar[kSbKFree + s], (n - 1) & 1, err, 0x401);
-                mbar_arrive_expect_tx(&bar[kSbKFull + s], kTileBytes);
-                tma_load_2d(sm + L::K0 + s * kTileBytes, &mk, 0, (int)(row0 + c * kTile),
-                            &bar[kSbKFull + s]);
-                if (n > 0) mbar_wait(&bar[kSbVFree + s], (n - 1) & 1, err, 0x402);
-                mbar_arrive_expect_tx(&bar[kSbVFull + s], kTileBytes);
-                tma_load_2d(sm + L::V0 + s * kTileBytes, &mv, 0, (int)(row0 + c * kTile),
-                            &bar[kSbVFull + s]);
+            // K and V tiles are freed by different consumers (the transposing
+            // workers, the MMAs): issue whichever slot frees first
+            int nk = 0, nv = 0;
+            uint32_t idle = 0;
+            while ((nk < p.nch || nv < p.nch) && idle < (1u << 24)) {
+                bool moved = false;
+                if (nk < p.nch) {
+                    const int ks = nk % L::KR, kn = nk / L::KR;
+                    if (kn == 0 || mbar_test_wait(&bar[kSbKFree + ks], (kn - 1) & 1)) {
+                        mbar_arrive_expect_tx(&bar[kSbKFull + ks], kTileBytes);
+                        tma_load_2d(sm + L::K0 + ks * kTileBytes, &mk, 0,
+                                    (int)(row0 + (long)nk * kTile), &bar[kSbKFull + ks]);
+                        ++nk;
+                        moved = true;
+                    }
+                }
+                if (nv < p.nch) {
+                    const int s = nv & 1, n = nv >> 1;
+                    if (n == 0 || mbar_test_wait(&bar[kSbVFree + s], (n - 1) & 1)) {
+                        mbar_arrive_expect_tx(&bar[kSbVFull + s], kTileBytes);
+                        tma_load_2d(sm + L::V0 + s * kTileBytes, &mv, 0,
+                                    (int)(row0 + (long)nv * kTile), &bar[kSbVFull + s]);
+                        ++nv;
+                        moved = true;
+                    }
+                }
+                if (!moved) {
+                    __nanosleep(32);
+                    if ((++idle & 1023u) == 0u && *((volatile unsigned int *)err) != 0u) break;
+                }
             }
+            if (nk < p.nch || nv < p.nch) atomicCAS(err, 0u, 0x401u);
             // no copy may still be in flight when the CTA exits
-            for (int c = p.nch - 2 < 0 ? 0 : p.nch - 2; c < p.nch; ++c) {
-                mbar_wait(&bar[kSbKFull + (c & 1)], (c >> 1) & 1, err, 0x403);
+            for (int c = p.nch - L::KR < 0 ? 0 : p.nch - L::KR; c < p.nch; ++c)
+                mbar_wait(&bar[kSbKFull + c % L::KR], (c / L::KR) & 1, err, 0x403);
+            for (int c = p.nch - 2 < 0 ? 0 : p.nch - 2; c < p.nch; ++c)
                 mbar_wait(&bar[kSbVFull + (c & 1)], (c >> 1) & 1, err, 0x404);
-            }
         }
-    } else if (warp == 4) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp >= 4) {
+        // ---------------- MMA issuer `ii`: K-steps ii, ii + NI, ... ----------------
+        const int ii = warp - 4;
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, kAccCols, 0, 1);
             const uint32_t ones = smem_u32(sm + L::ONES);
+            const uint32_t acc = tmem + L::acc_col(ii);
             for (int c = 0; c < p.nch; ++c) {
-                const int s = c & 1;
-                mbar_wait(&bar[kSbAFull + s], (c >> 1) & 1, err, 0x410);
+                const int s = c & 1, sa = c % NA;
+                mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412);
+                mbar_wait(&bar[kSbAFull + sa], (c / NA) & 1, err, 0x410);
                 // the state at an interval end must be read before it moves on
                 if (c > 0 && c % p.cpi == 0)
                     mbar_wait(&bar[kSbSnap], (c / p.cpi - 1) & 1, err, 0x411);
-                mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412);
                 tc_fence_after();
                 const uint32_t v = smem_u32(sm + L::V0 + s * kTileBytes);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    mma_ts(tmem + kStAcc, tmem + kStA + 64 * s + 8 * kk,
-                           vones_desc(v, ones, 16 * kk), idesc, 1);
+                for (int kk = ii; kk < kTile / 16; kk += NI)
+                    mma_ts(acc, tmem + L::A_COL + 64 * sa + 8 * kk, vones_desc(v, ones, 16 * kk),
+                           idesc, 1);
                 mma_commit(&bar[kSbVFree + s]);
-                mma_commit(&bar[kSbDone + s]);
+                mma_commit(&bar[kSbDone + sa]);
             }
         }
     } else {
@@ -262,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int slice = 2 * tile + (f >> 6);
         const bool valid = slice < S::NS;
+        const int nvalid = S::NS - 2 * tile < 2 ? S::NS - 2 * tile : 2;
         int ra = 0, rb = 0;
         if (valid) {
             int A, B;
@@ -270,16 +312,17 @@ __global__ void __launch_bounds__(kThreads, 2)
             rb = 8 * B + (f & 7);
         }
         uint8_t *kt = sm + L::KT;
+        uint8_t *stage = sm + L::STAGE;
 
-        // all-ones atom of the [V | 1] operand
+        // 16-row all-ones block of the [V | 1] operand
         {
             uint4 *o4 = reinterpret_cast<uint4 *>(sm + L::ONES);
-            for (int i = f; i < kTileBytes / 16; i += kWorkers)
+            for (int i = f; i < 2048 / 16; i += kWorkers)
                 o4[i] = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
             fence_proxy_async_smem();
         }
 
-        // initial state: H_in in the internal scaling (no sqrt 2), or zero
+        // initial state: H_in in the internal scaling (no sqrt 2) in accumulator 0
         float init[DH + 1];
         {
             const bool have = valid && p.H_in != nullptr;
@@ -298,82 +341,105 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const float x = col < DH ? init[col] : (col >= kSCol ? init[DH] : 0.f);
                     r[e] = __float_as_uint(x);
                 }
-                tmem_st16(tmem + lane_base + kStAcc + 16 * j, r);
+                tmem_st16(tmem + lane_base + L::acc_col(0) + 16 * j, r);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) r[e] = 0u;
+#pragma unroll
+                for (int i = 1; i < NI; ++i) tmem_st16(tmem + lane_base + L::acc_col(i) + 16 * j, r);
             }
             tmem_st_wait();
         }
-        // snapshot writer: rows n < DH take column n, rows DH.. take s
+        // snapshot: staged in shared memory as the readout's K-major operand
+        // (row n < DH = column n of H, rows DH.. = s), then one bulk store
+        // (thread 0 waits for the previous bulk store's read of the staging
+        // buffer before the first worker sync of each chunk)
         auto write_snapshot = [&](int g, const float (&x)[DH + 1]) {
-            if (!valid || p.snap == nullptr) return;
-            uint8_t *dst = p.snap +
-                           (((size_t)head * p.nint + g) * S::NS + slice) * S::SLICE_BYTES;
-            const int fl = f & 63;
+            if (p.snap == nullptr) return;
+            if (valid) {
+                uint8_t *row = stage + (f >> 6) * S::SLICE_BYTES;
+                const int fl = f & 63;
 #pragma unroll
-            for (int n = 0; n < S::NSNAP; ++n) {
-                const float val = n < DH ? x[n] : x[DH];
-                const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-                const uint32_t nb = __shfl_down_sync(0xFFFFFFFFu, h, 1);
-                if ((fl & 1) == 0)
-                    *reinterpret_cast<uint32_t *>(dst + n * 128 + (((fl >> 3) ^ (n & 7)) << 4) +
-                                                  (fl & 7) * 2) = h | (nb << 16);
+                for (int n = 0; n < S::NSNAP; ++n)
+                    *reinterpret_cast<__nv_bfloat16 *>(row + n * 128 +
+                                                       (((fl >> 3) ^ (n & 7)) << 4) +
+                                                       (fl & 7) * 2) =
+                        __float2bfloat16_rn(n < DH ? x[n] : x[DH]);
             }
+            fence_proxy_async_smem();
+            worker_sync();
+            if (f == 0)
+                bulk_store(p.snap + (((size_t)head * p.nint + g) * S::NS + 2 * tile) *
+                                        S::SLICE_BYTES,
+                           stage, nvalid * S::SLICE_BYTES);
         };
         if (p.H_in) write_snapshot(0, init);
-        // accumulator columns 0..DH-1 and the s column
+        if (f == 0) bulk_wait_read();
+        // the state: sum of the issuers' accumulators, columns 0..DH-1 and s
         auto read_acc = [&](float (&x)[DH + 1]) {
-            const uint32_t acc = tmem + lane_base + kStAcc;
 #pragma unroll
-            for (int j = 0; j < DH / 16; ++j) {
-                float y[16];
-                tmem_ld16_f(acc + 16 * j, y);
+            for (int n = 0; n <= DH; ++n) x[n] = 0.f;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) x[16 * j + e] = y[e];
+            for (int i = 0; i < NI; ++i) {
+                const uint32_t acc = tmem + lane_base + L::acc_col(i);
+                uint32_t r[DH / 16 + 1][16];
+#pragma unroll
+                for (int j = 0; j < DH / 16; ++j) tmem_ld16(acc + 16 * j, r[j]);
+                tmem_ld16(acc + kSCol, r[DH / 16]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < DH / 16; ++j)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x[16 * j + e] += __uint_as_float(r[j][e]);
+                x[DH] += __uint_as_float(r[DH / 16][0]);
             }
-            float y[16];
-            tmem_ld16_f(acc + kSCol, y);
-            x[DH] = y[0];
         };
 
+        constexpr int NCB = DH / 8;  // 8-column blocks of a K row
         for (int c = 0; c < p.nch; ++c) {
-            const int s = c & 1;
-            // transpose the K tile: thread = token
-            warp_wait(&bar[kSbKFull + s], (c >> 1) & 1, err, 0x420);
-            {
-                const uint8_t *kb = sm + L::K0 + s * kTileBytes;
-                const int t = f;
+            const int sa = c % NA, ks = c % L::KR;
+            // transpose the K tile in 8 x 8 blocks (8 tokens x 8 columns per thread)
+            warp_wait(&bar[kSbKFull + ks], (c / L::KR) & 1, err, 0x420);
+            if (f < 16 * NCB) {
+                const uint8_t *kb = sm + L::K0 + ks * kTileBytes;
+                const int tb = f / NCB, cb = f % NCB;
+                uint32_t x[8][4];
 #pragma unroll
-                for (int j = 0; j < DH / 8; ++j) {
-                    const uint4 x = *reinterpret_cast<const uint4 *>(kb + sw128_chunk(t, j));
-                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+                for (int r = 0; r < 8; ++r) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(kb + sw128_chunk(8 * tb + r, cb));
+                    x[r][0] = v.x;
+                    x[r][1] = v.y;
+                    x[r][2] = v.z;
+                    x[r][3] = v.w;
+                }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        *reinterpret_cast<uint16_t *>(kt + (8 * j + 2 * e) * kKtPitch + 2 * t) =
-                            (uint16_t)(w4[e] & 0xFFFFu);
-                        *reinterpret_cast<uint16_t *>(kt + (8 * j + 2 * e + 1) * kKtPitch + 2 * t) =
-                            (uint16_t)(w4[e] >> 16);
-                    }
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t sel = (cc & 1) ? 0x7632u : 0x5410u;
+                    uint4 y;
+                    y.x = __byte_perm(x[0][cc >> 1], x[1][cc >> 1], sel);
+                    y.y = __byte_perm(x[2][cc >> 1], x[3][cc >> 1], sel);
+                    y.z = __byte_perm(x[4][cc >> 1], x[5][cc >> 1], sel);
+                    y.w = __byte_perm(x[6][cc >> 1], x[7][cc >> 1], sel);
+                    *reinterpret_cast<uint4 *>(kt + kt_offset(8 * cb + cc, tb)) = y;
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kSbKFree + s]);
+            if (lane == 0) mbar_arrive(&bar[kSbKFree + ks]);
+            if (f == 0) bulk_wait_read();  // staging buffer free for the next snapshot
             worker_sync();  // K^T complete
             // Phi(K)^T row of feature (ra, rb): 128 tokens, two per 32-bit column
             uint32_t a_row[64];
-            {
-                const uint8_t *pa = kt + ra * kKtPitch, *pb = kt + rb * kKtPitch;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const uint4 x = *reinterpret_cast<const uint4 *>(pa + 16 * j);
-                    const uint4 y = *reinterpret_cast<const uint4 *>(pb + 16 * j);
-                    a_row[4 * j + 0] = valid ? hmul2(x.x, y.x) : 0u;
-                    a_row[4 * j + 1] = valid ? hmul2(x.y, y.y) : 0u;
-                    a_row[4 * j + 2] = valid ? hmul2(x.z, y.z) : 0u;
-                    a_row[4 * j + 3] = valid ? hmul2(x.w, y.w) : 0u;
-                }
+            for (int j = 0; j < 16; ++j) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(kt + kt_offset(ra, j));
+                const uint4 y = *reinterpret_cast<const uint4 *>(kt + kt_offset(rb, j));
+                a_row[4 * j + 0] = valid ? hmul2(x.x, y.x) : 0u;
+                a_row[4 * j + 1] = valid ? hmul2(x.y, y.y) : 0u;
+                a_row[4 * j + 2] = valid ? hmul2(x.z, y.z) : 0u;
+                a_row[4 * j + 3] = valid ? hmul2(x.w, y.w) : 0u;
             }
             worker_sync();  // K^T free for the next chunk
-            // A slot s was last read by chunk c - 2
-            if (c >= 2) warp_wait(&bar[kSbDone + s], ((c >> 1) - 1) & 1, err, 0x421);
+            // A slot sa was last read by chunk c - NA
+            if (c >= NA) warp_wait(&bar[kSbDone + sa], (c / NA - 1) & 1, err, 0x421);
             tc_fence_after();
             {
                 uint32_t r[16];
@@ -381,18 +447,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int j = 0; j < 4; ++j) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) r[e] = a_row[16 * j + e];
-                    tmem_st16(tmem + lane_base + kStA + 64 * s + 16 * j, r);
+                    tmem_st16(tmem + lane_base + L::A_COL + 64 * sa + 16 * j, r);
                 }
                 tmem_st_wait();
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kSbAFull + s]);
+            if (lane == 0) mbar_arrive(&bar[kSbAFull + sa]);
             // chunk c opens interval g: the state after chunk c - 1 is snapshot g
-            // (A(c) is already published, so the issuer waits only for this read)
+            // (A(c) is already published, so the issuers wait only for this read)
             if (c > 0 && c % p.cpi == 0) {
-                const int sp = (c - 1) & 1;
-                warp_wait(&bar[kSbDone + sp], ((c - 1) >> 1) & 1, err, 0x422);
+                warp_wait(&bar[kSbDone + (c - 1) % NA], ((c - 1) / NA) & 1, err, 0x422);
                 tc_fence_after();
                 float x[DH + 1];
                 read_acc(x);
@@ -403,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         // final state, converted to the canonical layout
-        warp_wait(&bar[kSbDone + ((p.nch - 1) & 1)], ((p.nch - 1) >> 1) & 1, err, 0x423);
+        warp_wait(&bar[kSbDone + (p.nch - 1) % NA], ((p.nch - 1) / NA) & 1, err, 0x423);
         tc_fence_after();
         if (p.H_out) {
             float fin[DH + 1];
@@ -420,13 +485,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 p.s_out[hb] = fin[DH] * w;
             }
         }
+        if (f == 0) bulk_wait_all();
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 4) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, L::TMEM_COLS);
     }
 }
 
@@ -469,8 +535,8 @@ struct ReadSmem {
     static constexpr int Q = 0;
     static constexpr int K = kTileBytes;
     static constexpr int V = 2 * kTileBytes;
-    static constexpr int ONES = 3 * kTileBytes;
-    static constexpr int P = 4 * kTileBytes;  // kRP snapshot slices
+    static constexpr int ONES = 3 * kTileBytes;   // 16-row all-ones block
+    static constexpr int P = 3 * kTileBytes + 2048;  // kRP snapshot slices
     static constexpr int BAR = P + kRP * Shape<DH>::SLICE_BYTES;
     static constexpr int SLOT = BAR + kRbCount * 8;
     static constexpr int BYTES = SLOT + 16 + 1024;
@@ -622,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; j < kAccCols / 16; ++j) tmem_st16(tmem + lane_base + kRdO + 16 * j, z);
             tmem_st_wait();
             uint4 *o4 = reinterpret_cast<uint4 *>(sm + L::ONES);
-            for (int x = i; x < kTileBytes / 16; x += kWorkers)
+            for (int x = i; x < 2048 / 16; x += kWorkers)
                 o4[x] = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
             fence_proxy_async_smem();
         }
@@ -761,7 +827,7 @@ bool make_map(CUtensorMap *m, const void *base, int d, long rows) {
 // Chunks per snapshot interval: longer intervals mean fewer snapshot bytes
 // and more quadratic intra work per query tile.
 int chunks_per_interval(int d, int nch) {
-    int c = d == 64 ? 4 : 1;
+    int c = d == 64 ? 4 : 2;
     while (c > 1 && nch % c) c >>= 1;
     return c;
 }
@@ -788,12 +854,13 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
 
     StateParams sp{nch, cpi, nint, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
     {
-        auto kern = state_kernel<DH>;
-        const int bytes = StateSmem<DH>::BYTES;
+        // two issuers (one Phi(K)^T slot) halve the MMA issue chain of a chunk
+        using L = StateCfg<DH, 2, 1>;
+        auto kern = state_kernel<DH, 2, 1>;
         cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
         if (e != cudaSuccess) return e;
-        kern<<<dim3(S::NT, nheads), kThreads, bytes, stream>>>(mk, mv, sp);
+        kern<<<dim3(S::NT, nheads), L::THREADS, L::BYTES, stream>>>(mk, mv, sp);
         e = after_launch();
         if (e != cudaSuccess) return e;
     }

@@ -66,10 +66,27 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 
+// Non-blocking probe of the phase with this parity (try_wait may suspend the
+// thread for a while; a thread that polls several barriers uses this).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: returns false (and records `code` in *err) if the phase with
-// this parity has not completed after `limit` polls.
+// this parity has not completed after `limit` polls. A phase that has already
+// completed is seen by the cheap non-blocking probe; only a wait that has to
+// wait uses the suspending form.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
                                           unsigned int code, uint32_t limit = 1u << 22) {
+    if (mbar_test_wait(bar, parity)) return true;
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if (err && (i & 1023u) == 1023u && *((volatile unsigned int *)err) != 0u) return false;
@@ -119,6 +136,24 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
             "r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Contiguous shared -> global copy, tracked by the issuing thread's bulk
+// group; same alignment rules as bulk_load.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(dst)),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The source shared memory of this thread's earlier bulk stores may be reused.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's earlier bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
