@@ -32,12 +32,11 @@
 // sqrt(2) of the canonical packed layout; kata_prefill's H_in/H_out use the
 // canonical one and the state kernel converts at both ends.
 //
-// Column layout of the fp32 accumulators (state and output): columns 0..d-1
-// hold H (or the numerator), columns 64..79 all hold s (or the denominator)
-// because the [V | 1] operand is the V tile followed by a 64-wide all-ones
-// block; for d = 32 columns 32..63 are zero. The snapshot slices hold rows
-// 0..d-1 = H and d..d+15 = s, so the inter MMA writes the denominator part to
-// column d: the readout sums columns d and 64 (the same column for d = 64).
+// Column layout of the fp32 accumulators (state and output), N = d + 16
+// columns: 0..d-1 hold H (or the numerator), d..d+15 all hold s (or the
+// denominator), because the [V | 1] operand is the V tile (one swizzle atom of
+// d columns: 128-byte swizzle for d = 64, 64-byte for d = 32) followed by an
+// all-ones block. The snapshot slices hold rows 0..d-1 = H and d..d+15 = s.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -55,10 +54,7 @@ using namespace sm100;
 
 constexpr int kTile = 128;         // tokens per chunk / query tile; rows per state tile
 constexpr int kTileBytes = 16384;  // one 128 x 64 bf16 tile, 128-byte swizzle
-constexpr int kAccCols = 80;       // accumulator columns: H (<= 64) | s x 16
-constexpr int kSCol = 64;          // first accumulator column holding s
 constexpr int kWorkers = 128;      // 4 warps: one thread per tensor-memory lane
-constexpr int kThreads = 192;      // + MMA issuer warp + TMA producer warp
 constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
 
 template <int DH>
@@ -68,6 +64,12 @@ struct Shape {
     static constexpr int NT = (NS + 1) / 2;       // 128-row state tiles
     static constexpr int NSNAP = DH + 16;         // snapshot rows: H | s x 16
     static constexpr int SLICE_BYTES = NSNAP * 128;
+    static constexpr int NACC = DH + 16;          // accumulator columns: H | s x 16
+    static constexpr int SCOL = DH;               // first accumulator column holding s
+    static constexpr int ACC_PITCH = DH == 64 ? 96 : 64;  // tensor-memory columns per accumulator
+    static constexpr int VROW = 2 * DH;           // bytes per V row (one swizzle atom)
+    static constexpr int VBYTES = kTile * VROW;
+    static constexpr uint32_t VSW = DH == 64 ? kSwizzle128 : kSwizzle64;
 };
 
 // Block pair (A, B), A <= B, of slice s: slices run A-major, B ascending.
@@ -114,21 +116,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsign
     return ok != 0;
 }
 
-__device__ __forceinline__ void tmem_ld16_f(uint32_t taddr, float (&f)[16]) {
-    uint32_t r[16];
-    tmem_ld16(taddr, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(r[e]);
-}
-
 // MN-major [V | 1] operand for 16 tokens starting at row `row0` of the V tile:
-// the V tile (64 bf16 per row, zero-filled past d) is the first 64-column
-// atom; the second atom is a 16-row all-ones block, reached through the
-// leading byte offset from this K-step's start (every row of it is the same).
+// the V tile (d bf16 per row) is the first atom; the second atom is a 16-row
+// all-ones block, reached through the leading byte offset from this K-step's
+// start (every row of it is the same).
+template <int DH>
 __device__ __forceinline__ uint64_t vones_desc(uint32_t v, uint32_t ones, int row0) {
-    const uint32_t start = v + row0 * 128;
-    return smem_desc(start, ones - start, 1024, kSwizzle128);
+    using S = Shape<DH>;
+    const uint32_t start = v + row0 * S::VROW;
+    return smem_desc(start, ones - start, 8 * S::VROW, S::VSW);
 }
 
 // K-major operand: 128-byte rows, 16 K-elements at byte offset 32 * kk.
@@ -174,17 +170,19 @@ struct StateCfg {
     static constexpr int KR = DH == 64 ? 2 : 3;  // K tiles in flight
     static constexpr int K0 = 0;
     static constexpr int V0 = KR * kTileBytes;    // 2 x V tile
-    static constexpr int ONES = V0 + 2 * kTileBytes;
+    static constexpr int ONES = V0 + 2 * Shape<DH>::VBYTES;
     static constexpr int KT = ONES + 2048;
     static constexpr int STAGE = KT + DH * 256;   // snapshot staging: 2 slices
     static constexpr int BAR = STAGE + 2 * Shape<DH>::SLICE_BYTES;
     static constexpr int SLOT = BAR + kSbCount * 8;
     static constexpr int BYTES = SLOT + 16 + 1024;
     static constexpr int THREADS = 32 * (5 + NI);  // workers, NI issuers, TMA
-    // NI accumulators of 80 columns at a 96-column pitch, then NA Phi(K)^T slots
-    static constexpr uint32_t A_COL = 96u * NI;
+    // NI accumulators, then NA Phi(K)^T slots of 64 columns
+    static constexpr uint32_t A_COL = (NI * Shape<DH>::ACC_PITCH + 63) / 64 * 64;
     static constexpr uint32_t TMEM_COLS = A_COL + 64u * NA <= 256 ? 256 : 512;
-    __host__ __device__ static constexpr uint32_t acc_col(int i) { return 96u * i; }
+    __host__ __device__ static constexpr uint32_t acc_col(int i) {
+        return (uint32_t)(Shape<DH>::ACC_PITCH * i);
+    }
 };
 
 template <int DH, int NI, int NA>
@@ -254,8 +252,8 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 if (nv < p.nch) {
                     const int s = nv & 1, n = nv >> 1;
                     if (n == 0 || mbar_test_wait(&bar[kSbVFree + s], (n - 1) & 1)) {
-                        mbar_arrive_expect_tx(&bar[kSbVFull + s], kTileBytes);
-                        tma_load_2d(sm + L::V0 + s * kTileBytes, &mv, 0,
+                        mbar_arrive_expect_tx(&bar[kSbVFull + s], S::VBYTES);
+                        tma_load_2d(sm + L::V0 + s * S::VBYTES, &mv, 0,
                                     (int)(row0 + (long)nv * kTile), &bar[kSbVFull + s]);
                         ++nv;
                         moved = true;
@@ -277,7 +275,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
         // ---------------- MMA issuer `ii`: K-steps ii, ii + NI, ... ----------------
         const int ii = warp - 4;
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, kAccCols, 0, 1);
+            const uint32_t idesc = idesc_bf16(128, S::NACC, 0, 1);
             const uint32_t ones = smem_u32(sm + L::ONES);
             const uint32_t acc = tmem + L::acc_col(ii);
             for (int c = 0; c < p.nch; ++c) {
@@ -288,11 +286,11 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 if (c > 0 && c % p.cpi == 0)
                     mbar_wait(&bar[kSbSnap], (c / p.cpi - 1) & 1, err, 0x411);
                 tc_fence_after();
-                const uint32_t v = smem_u32(sm + L::V0 + s * kTileBytes);
+                const uint32_t v = smem_u32(sm + L::V0 + s * S::VBYTES);
 #pragma unroll
                 for (int kk = ii; kk < kTile / 16; kk += NI)
-                    mma_ts(acc, tmem + L::A_COL + 64 * sa + 8 * kk, vones_desc(v, ones, 16 * kk),
-                           idesc, 1);
+                    mma_ts(acc, tmem + L::A_COL + 64 * sa + 8 * kk,
+                           vones_desc<DH>(v, ones, 16 * kk), idesc, 1);
                 mma_commit(&bar[kSbVFree + s]);
                 mma_commit(&bar[kSbDone + sa]);
             }
@@ -334,12 +332,11 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             init[DH] = have ? p.s_in[hb] * w : 0.f;
             uint32_t r[16];
 #pragma unroll
-            for (int j = 0; j < kAccCols / 16; ++j) {
+            for (int j = 0; j < S::NACC / 16; ++j) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int col = 16 * j + e;
-                    const float x = col < DH ? init[col] : (col >= kSCol ? init[DH] : 0.f);
-                    r[e] = __float_as_uint(x);
+                    r[e] = __float_as_uint(col < DH ? init[col] : init[DH]);
                 }
                 tmem_st16(tmem + lane_base + L::acc_col(0) + 16 * j, r);
 #pragma unroll
@@ -384,7 +381,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 uint32_t r[DH / 16 + 1][16];
 #pragma unroll
                 for (int j = 0; j < DH / 16; ++j) tmem_ld16(acc + 16 * j, r[j]);
-                tmem_ld16(acc + kSCol, r[DH / 16]);
+                tmem_ld16(acc + S::SCOL, r[DH / 16]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < DH / 16; ++j)
@@ -500,8 +497,8 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
 // Readout kernel
 // ---------------------------------------------------------------------------
 
-constexpr int kRP = 4;  // snapshot slices in flight
-constexpr int kRQ = 3;  // A-operand slots in tensor memory
+constexpr int kRP = 4;      // snapshot slices in flight
+constexpr int kRQMax = 3;   // A-operand slots in tensor memory (at most)
 
 struct ReadParams {
     int nch;     // query tiles (= chunks) per head
@@ -526,12 +523,12 @@ enum ReadBar {
     kRbPFull = 8,
     kRbPFree = kRbPFull + kRP,
     kRbAqFull = kRbPFree + kRP,  // 4 warp arrivals
-    kRbAqFree = kRbAqFull + kRQ,
-    kRbCount = kRbAqFree + kRQ
+    kRbAqFree = kRbAqFull + kRQMax,
+    kRbCount = kRbAqFree + kRQMax
 };
 
-template <int DH>
-struct ReadSmem {
+template <int DH, int NIR>
+struct ReadCfg {
     static constexpr int Q = 0;
     static constexpr int K = kTileBytes;
     static constexpr int V = 2 * kTileBytes;
@@ -540,17 +537,28 @@ struct ReadSmem {
     static constexpr int BAR = P + kRP * Shape<DH>::SLICE_BYTES;
     static constexpr int SLOT = BAR + kRbCount * 8;
     static constexpr int BYTES = SLOT + 16 + 1024;
+    static constexpr int THREADS = 32 * (5 + NIR);  // workers, NIR issuers, TMA
+    static constexpr int TMA_WARP = 4 + NIR;
+    // tensor memory (256 columns): NIR output accumulators, S (64 keys), then
+    // RQ A-operand slots of 32 columns
+    static constexpr uint32_t S_COL = (NIR * Shape<DH>::ACC_PITCH + 31) / 32 * 32;
+    static constexpr uint32_t AQ_COL = S_COL + 64;
+    static constexpr int RQ = (256 - AQ_COL) / 32 < kRQMax ? (256 - AQ_COL) / 32 : kRQMax;
+    __host__ __device__ static constexpr uint32_t o_col(int i) {
+        return (uint32_t)(Shape<DH>::ACC_PITCH * i);
+    }
+    static_assert(RQ >= 2 && RQ % NIR == 0, "tensor-memory budget");
+    // every snapshot slot is consumed by one issuer only (slices s, s + kRP, ...)
+    static_assert(kRP % NIR == 0, "snapshot ring must divide among the issuers");
 };
 
-// Tensor-memory columns of the readout kernel (256 allocated).
-constexpr uint32_t kRdO = 0, kRdS = 96, kRdAq = 160;
-
-template <int DH>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int DH, int NIR>
+__global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
     readout_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                    const __grid_constant__ CUtensorMap mv, ReadParams p) {
     using S = Shape<DH>;
-    using L = ReadSmem<DH>;
+    using L = ReadCfg<DH, NIR>;
+    constexpr int RQ = L::RQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -560,17 +568,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int m = blockIdx.x, head = blockIdx.y;  // query tile, (batch, head)
     unsigned int *err = p.err;
 
-    const int g = m / p.cpi;             // snapshot interval of this query tile
-    const int kt0 = g * p.cpi;           // first key tile of the interval
+    const int g = m / p.cpi;               // snapshot interval of this query tile
+    const int kt0 = g * p.cpi;             // first key tile of the interval
     const int n_half = 2 * (m - kt0 + 1);  // intra items: 64-key halves
     const int n_inter = (g > 0 || p.has_in) ? S::NS : 0;
     const int n_items = n_half + n_inter;
     const long row0 = (long)head * p.nch * kTile;
+    // item -> issuer: the intra items (and S) on issuer 0, inter slices round-robin.
+    // Each issuer owns SPI of the A-operand slots, so every slot's barriers are
+    // consumed in phase order by one issuer (a parity wait only tells the
+    // current phase from the one before it).
+    constexpr int SPI = RQ / NIR;
+    auto issuer_of = [&](int it) { return it < n_half ? 0 : (it - n_half) % NIR; };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kRbCount; ++i) {
-            const bool four = i == kRbSFree || (i >= kRbAqFull && i < kRbAqFull + kRQ);
-            mbar_init(&bar[i], four ? 4 : 1);
+            const bool four = i == kRbSFree || (i >= kRbAqFull && i < kRbAqFull + kRQMax);
+            mbar_init(&bar[i], four ? 4 : (i == kRbODone ? NIR : 1));
         }
         fence_barrier_init();
     }
@@ -585,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint8_t *snap =
         p.snap + ((size_t)head * p.nint + g) * S::NS * (size_t)S::SLICE_BYTES;
 
-    if (warp == 5) {
+    if (warp == L::TMA_WARP) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&mq);
@@ -604,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive_expect_tx(&bar[kRbKFull], kTileBytes);
                 tma_load_2d(sm + L::K, &mk, 0, y, &bar[kRbKFull]);
                 if (u > 0) mbar_wait(&bar[kRbVFree], (u - 1) & 1, err, 0x503);
-                mbar_arrive_expect_tx(&bar[kRbVFull], kTileBytes);
+                mbar_arrive_expect_tx(&bar[kRbVFull], S::VBYTES);
                 tma_load_2d(sm + L::V, &mv, 0, y, &bar[kRbVFull]);
             };
             mbar_arrive_expect_tx(&bar[kRbQFull], kTileBytes);
@@ -622,53 +636,61 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int s = n_inter - kRP < 0 ? 0 : n_inter - kRP; s < n_inter; ++s)
                 mbar_wait(&bar[kRbPFull + s % kRP], (s / kRP) & 1, err, 0x507);
         }
-    } else if (warp == 4) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp >= 4) {
+        // ---------------- MMA issuer `ii` ----------------
+        const int ii = warp - 4;
         if (lane == 0) {
             const uint32_t i_s = idesc_bf16(128, 64, 0, 0);
-            const uint32_t i_av = idesc_bf16(128, kAccCols, 0, 1);
+            const uint32_t i_av = idesc_bf16(128, S::NACC, 0, 1);
             const uint32_t i_p = idesc_bf16(128, S::NSNAP, 0, 0);
             const uint32_t q_a = smem_u32(sm + L::Q), k_a = smem_u32(sm + L::K);
             const uint32_t v_a = smem_u32(sm + L::V), ones = smem_u32(sm + L::ONES);
+            const uint32_t o_acc = tmem + L::o_col(ii);
             auto issue_s = [&](int j) {  // S = Q K^T for 64-key half j
                 const int u = j >> 1, h = j & 1;
                 if (h == 0) mbar_wait(&bar[kRbKFull], u & 1, err, 0x510);
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk)
-                    mma_ss(tmem + kRdS, kmaj_desc(q_a, kk), kmaj_desc(k_a + h * 64 * 128, kk), i_s,
-                           kk > 0);
+                    mma_ss(tmem + L::S_COL, kmaj_desc(q_a, kk), kmaj_desc(k_a + h * 64 * 128, kk),
+                           i_s, kk > 0);
                 mma_commit(&bar[kRbSFull]);
                 if (h == 1) mma_commit(&bar[kRbKFree]);
             };
-            mbar_wait(&bar[kRbQFull], 0, err, 0x511);
-            issue_s(0);
+            if (ii == 0) {
+                mbar_wait(&bar[kRbQFull], 0, err, 0x511);
+                issue_s(0);
+            }
+            int uses = 0;  // this issuer's items so far
             for (int it = 0; it < n_items; ++it) {
-                const int slot = it % kRQ;
+                if (issuer_of(it) != ii) continue;
+                const int u = uses++;
+                const int slot = ii * SPI + u % SPI;
+                const uint32_t ph = (uint32_t)(u / SPI) & 1u;
                 if (it < n_half) {
                     const int j = it, h = j & 1;
                     if (j + 1 < n_half) {
                         mbar_wait(&bar[kRbSFree], j & 1, err, 0x512);
                         issue_s(j + 1);
                     }
-                    mbar_wait(&bar[kRbAqFull + slot], (it / kRQ) & 1, err, 0x513);
+                    mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x513);
                     if (h == 0) mbar_wait(&bar[kRbVFull], (j >> 1) & 1, err, 0x514);
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + kRdO, tmem + kRdAq + 32 * slot + 8 * kk,
-                               vones_desc(v_a, ones, 64 * h + 16 * kk), i_av, 1);
+                        mma_ts(o_acc, tmem + L::AQ_COL + 32 * slot + 8 * kk,
+                               vones_desc<DH>(v_a, ones, 64 * h + 16 * kk), i_av, 1);
                     mma_commit(&bar[kRbAqFree + slot]);
                     if (h == 1) mma_commit(&bar[kRbVFree]);
                 } else {
                     const int s = it - n_half, ps = s % kRP;
-                    mbar_wait(&bar[kRbAqFull + slot], (it / kRQ) & 1, err, 0x515);
                     mbar_wait(&bar[kRbPFull + ps], (s / kRP) & 1, err, 0x516);
+                    mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x515);
                     tc_fence_after();
                     const uint32_t pa = smem_u32(sm + L::P + ps * S::SLICE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + kRdO, tmem + kRdAq + 32 * slot + 8 * kk, kmaj_desc(pa, kk),
+                        mma_ts(o_acc, tmem + L::AQ_COL + 32 * slot + 8 * kk, kmaj_desc(pa, kk),
                                i_p, 1);
                     mma_commit(&bar[kRbAqFree + slot]);
                     mma_commit(&bar[kRbPFree + ps]);
@@ -685,7 +707,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int e = 0; e < 16; ++e) z[e] = 0u;
 #pragma unroll
-            for (int j = 0; j < kAccCols / 16; ++j) tmem_st16(tmem + lane_base + kRdO + 16 * j, z);
+            for (int a = 0; a < NIR; ++a)
+#pragma unroll
+                for (int j = 0; j < S::NACC / 16; ++j)
+                    tmem_st16(tmem + lane_base + L::o_col(a) + 16 * j, z);
             tmem_st_wait();
             uint4 *o4 = reinterpret_cast<uint4 *>(sm + L::ONES);
             for (int x = i; x < 2048 / 16; x += kWorkers)
@@ -693,8 +718,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             fence_proxy_async_smem();
         }
         warp_wait(&bar[kRbQFull], 0, err, 0x520);
+        int uses0 = 0, uses1 = 0;  // items so far of issuer 0 and issuer 1
         for (int it = 0; it < n_items; ++it) {
-            const int slot = it % kRQ;
+            const int iss = issuer_of(it);
+            const int u = iss == 0 ? uses0++ : uses1++;
+            const int slot = iss * SPI + u % SPI;
             uint32_t pk[32];
             if (it < n_half) {
                 // intra: squared scores of 64 keys, causal mask on the diagonal tile
@@ -706,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t r[16];
-                    tmem_ld16(tmem + lane_base + kRdS + 16 * q4, r);
+                    tmem_ld16(tmem + lane_base + L::S_COL + 16 * q4, r);
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sv[16 * q4 + e] = __uint_as_float(r[e]);
                 }
@@ -739,47 +767,47 @@ __global__ void __launch_bounds__(kThreads, 2)
                     for (int bb = 0; bb < 4; ++bb) pk[4 * a + bb] = hmul2(qa, wb[bb]);
                 }
             }
-            if (it >= kRQ) warp_wait(&bar[kRbAqFree + slot], ((it / kRQ) - 1) & 1, err, 0x522);
+            if (u >= SPI) warp_wait(&bar[kRbAqFree + slot], (u / SPI - 1) & 1, err, 0x522);
             tc_fence_after();
             {
                 uint32_t r[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) r[e] = pk[e];
-                tmem_st16(tmem + lane_base + kRdAq + 32 * slot, r);
+                tmem_st16(tmem + lane_base + L::AQ_COL + 32 * slot, r);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) r[e] = pk[16 + e];
-                tmem_st16(tmem + lane_base + kRdAq + 32 * slot + 16, r);
+                tmem_st16(tmem + lane_base + L::AQ_COL + 32 * slot + 16, r);
             }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[kRbAqFull + slot]);
         }
-        // epilogue: o = numerator / (denominator + eps)
+        // epilogue: o = numerator / (denominator + eps), summed over the issuers
         warp_wait(&bar[kRbODone], 0, err, 0x523);
         tc_fence_after();
-        float den;
-        {
-            float x[16];
-            tmem_ld16_f(tmem + lane_base + kRdO + kSCol, x);
-            den = x[0];
-            if (DH < kSCol) {
-                tmem_ld16_f(tmem + lane_base + kRdO + DH, x);
-                den += x[0];
-            }
+        float num[DH], den = 0.f;
+#pragma unroll
+        for (int n = 0; n < DH; ++n) num[n] = 0.f;
+#pragma unroll
+        for (int a = 0; a < NIR; ++a) {
+            uint32_t r[DH / 16 + 1][16];
+#pragma unroll
+            for (int j = 0; j <= DH / 16; ++j) tmem_ld16(tmem + lane_base + L::o_col(a) + 16 * j, r[j]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < DH / 16; ++j)
+#pragma unroll
+                for (int e = 0; e < 16; ++e) num[16 * j + e] += __uint_as_float(r[j][e]);
+            den += __uint_as_float(r[DH / 16][0]);
         }
         const float inv = 1.f / (den + p.eps);
         float4 *dst =
             reinterpret_cast<float4 *>(p.o + ((size_t)head * p.nch * kTile + (size_t)m * kTile + i) * DH);
 #pragma unroll
-        for (int j = 0; j < DH / 16; ++j) {
-            float x[16];
-            tmem_ld16_f(tmem + lane_base + kRdO + 16 * j, x);
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                dst[4 * j + e / 4] = make_float4(x[e] * inv, x[e + 1] * inv, x[e + 2] * inv,
-                                                 x[e + 3] * inv);
-        }
+        for (int n = 0; n < DH; n += 4)
+            dst[n / 4] = make_float4(num[n] * inv, num[n + 1] * inv, num[n + 2] * inv,
+                                     num[n + 3] * inv);
     }
 
     tc_fence_before();
@@ -808,19 +836,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// [rows, d] bf16 rows, 128 x 64 boxes with the 128-byte swizzle; for d = 32
-// the box reaches past the row and the extra columns are zero-filled.
-bool make_map(CUtensorMap *m, const void *base, int d, long rows) {
+// [rows, d] bf16 rows in boxes of 128 rows x box_x columns. Q and K use
+// box_x = 64 with the 128-byte swizzle (for d = 32 the box reaches past the row
+// and the extra columns are zero-filled); V uses box_x = d, one swizzle atom
+// (128-byte swizzle for d = 64, 64-byte for d = 32).
+bool make_map(CUtensorMap *m, const void *base, int d, long rows, int box_x,
+              CUtensorMapSwizzle sw) {
     auto enc = get_encode();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)kTile};
     cuuint32_t es[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -848,15 +878,20 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     uint8_t *snap = want_o ? static_cast<uint8_t *>(a.ws) : nullptr;
     if (want_o && a.ws_bytes < snapshot_bytes<DH>(nheads, nch)) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, DH, rows) || !make_map(&mk, a.k, DH, rows) ||
-        !make_map(&mv, a.v, DH, rows))
+    const CUtensorMapSwizzle vsw =
+        DH == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!make_map(&mq, a.q, DH, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mk, a.k, DH, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mv, a.v, DH, rows, DH, vsw))
         return cudaErrorInvalidValue;
 
     StateParams sp{nch, cpi, nint, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
     {
-        // two issuers (one Phi(K)^T slot) halve the MMA issue chain of a chunk
-        using L = StateCfg<DH, 2, 1>;
-        auto kern = state_kernel<DH, 2, 1>;
+        // two issuers halve the MMA issue chain of a chunk; with d = 32 the
+        // accumulators are narrow enough to keep two Phi(K)^T slots as well
+        constexpr int NA = DH == 64 ? 1 : 2;
+        using L = StateCfg<DH, 2, NA>;
+        auto kern = state_kernel<DH, 2, NA>;
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
         if (e != cudaSuccess) return e;
@@ -866,11 +901,13 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     }
     if (!want_o) return cudaSuccess;
     ReadParams rp{nch, cpi, nint, a.H_in != nullptr ? 1 : 0, snap, a.o, a.eps, a.err};
-    auto kern = readout_kernel<DH>;
-    const int bytes = ReadSmem<DH>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // two issuers where the accumulators leave room for them (d = 32)
+    constexpr int NIR = DH == 64 ? 1 : 2;
+    using R = ReadCfg<DH, NIR>;
+    auto kern = readout_kernel<DH, NIR>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, R::BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(nch, nheads), kThreads, bytes, stream>>>(mq, mk, mv, rp);
+    kern<<<dim3(nch, nheads), R::THREADS, R::BYTES, stream>>>(mq, mk, mv, rp);
     return after_launch();
 }
 

@@ -271,6 +271,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 
 constexpr uint32_t kSwizzle128 = 2;
+constexpr uint32_t kSwizzle64 = 4;
 
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulate.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
