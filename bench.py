@@ -52,6 +52,12 @@ def prefill_flops(w) -> float:
     return float(per) * w.B * w.H * w.T
 
 
+def prefill_update_flops(w) -> float:
+    """The state-update half of the inter-chunk flops: 2 D (d+1) per head-token."""
+    D = w.d * (w.d + 1) // 2
+    return float(2 * D * (w.d + 1)) * w.B * w.H * w.T
+
+
 def prefill_bytes(w) -> float:
     """Compulsory HBM bytes: q, k, v in, o (fp32) out."""
     es = 2 if w.dtype == "bf16" else 4
@@ -301,28 +307,61 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     flops = prefill_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
 
-    # roofline of the dominant kernel: the prefill kernel, one launch per call
+    # roofline of the dominant kernel. The tensor-core path is two launches per
+    # call: the state kernel (chunk-state accumulation and carry, half the
+    # inter-chunk flops) and the readout kernel (the other half plus the
+    # intra-chunk part). The state kernel is timed alone by a state-only call
+    # (it then writes the final state instead of the snapshots); the readout is
+    # the difference.
     lat = per_launch_ms(step, max(args.steps, 5), stream)
     path = "tc" if kata.prefill_uses_tensor_cores(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16) \
         else "simt"
+    kernels = None
     if path == "tc":
-        roof = {"bound": "tensor", "achieved": flops / (lat / 1e3) / 1e12,
+        Hs = torch.empty(w.B, w.H, w.D, w.d, device=dev)
+        ss = torch.empty(w.B, w.H, w.D, device=dev)
+
+        def state_step(i):
+            qq, kk, vv = sets[i % R]
+            kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, output=False, H_out=Hs,
+                         s_out=ss, workspace=ws)
+
+        for i in range(3):
+            state_step(i)
+        lat_state = per_launch_ms(state_step, max(args.steps, 5), stream)
+        lat_read = max(lat - lat_state, 1e-6)
+        f_update = prefill_update_flops(w)
+        f_read = flops - f_update
+        kernels = {
+            "state_kernel": {"ms": lat_state, "tflops": f_update / (lat_state / 1e3) / 1e12},
+            "readout_kernel": {"ms": lat_read, "tflops": f_read / (lat_read / 1e3) / 1e12,
+                               "note": "call time minus the state-only call"}}
+        dom = "state_kernel" if lat_state >= lat_read else "readout_kernel"
+        dom_ms = lat_state if dom == "state_kernel" else lat_read
+        dom_flops = f_update if dom == "state_kernel" else f_read
+        roof = {"bound": "tensor", "achieved": dom_flops / (dom_ms / 1e3) / 1e12,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        kernel = "prefill_tc_kernel"
+        kernel = dom
+        del Hs, ss
     else:
         # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x max SM clock
         alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof = {"bound": "alu", "achieved": flops / (lat / 1e3) / 1e12, "peak": alu_peak,
                 "unit": "TFLOP/s"}
         kernel = "prefill_simt_kernel"
+        dom_ms = lat
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
     roof["kernel"] = kernel
-    roof["launch_ms"] = lat
+    roof["launch_ms"] = dom_ms
     roof["traffic"] = traffic_record(kernel, HEADLINE)
+    roof["call_ms"] = lat
+    roof["call_tflops"] = flops / (lat / 1e3) / 1e12
     roof["algorithmic_bytes"] = prefill_bytes(w)
-    roof["hbm_frac"] = prefill_bytes(w) / (lat / 1e3) / 1e9 / peaks["hbm_gbs"]
+    roof["call_hbm_frac"] = prefill_bytes(w) / (lat / 1e3) / 1e9 / peaks["hbm_gbs"]
+    if kernels:
+        roof["kernels"] = kernels
 
     # end to end: host q, k, v in, host o out, through the C ABI
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
