@@ -35,7 +35,7 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 from kernelized_linear_attention_chunked_b200.inputs import (  # noqa: E402
-    WORKLOADS, decode_inputs, prefill_inputs, recall_inputs)
+    WORKLOADS, candidate_inputs, decode_inputs, prefill_inputs, recall_inputs)
 
 METRIC = "prefill tokens/s & TFLOP/s (% bf16 peak); decode tokens/s (% HBM BW), 1×B200"
 HEADLINE = "prefill_b4_h8_t2048_d32"
@@ -254,7 +254,9 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
         fn = {"decode": lambda: bench_decode(kata, args, dev, stream, peaks, dist_on, world),
               "long_prefill": lambda: bench_long_prefill(kata, args, dev, stream, peaks,
                                                          dist_on, world),
-              "lola": lambda: bench_lola(kata, args, dev, stream, dist_on, world)}[args.only]
+              "lola": lambda: bench_lola(kata, args, dev, stream, dist_on, world),
+              "sre_stress": lambda: bench_sre_stress(kata, args, dev, stream, peaks, dist_on,
+                                                     world)}[args.only]
         res = fn()
         if rank == 0:
             print(json.dumps({"only": args.only, args.only: res}), flush=True)
@@ -387,6 +389,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
         sub["decode"] = bench_decode(kata, args, dev, stream, peaks, dist_on, world)
         sub["long_prefill"] = bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world)
         sub["lola"] = bench_lola(kata, args, dev, stream, dist_on, world)
+        sub["sre_stress"] = bench_sre_stress(kata, args, dev, stream, peaks, dist_on, world)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -438,6 +441,48 @@ def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
             "us_per_step": 1e3 * ms_step, "steps": nsteps, "gbs": gbs,
             "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_step": decode_bytes(w),
             "gpu_launches": launches, "l2": "state 554 MB > 126 MB L2"}
+
+
+def bench_sre_stress(kata, args, dev, stream, peaks, dist_on, world):
+    """One SRE score + top-k + merge pass over a state larger than L2: B64 H16
+    d64 (553.8 MB fp32 state), 192 candidates per head, keep 128, the other 64
+    merged in place. The state is seeded normal values (scale 0.01) with a
+    positive normaliser; candidates come from the seeded candidate generator.
+    Algorithmic bytes per pass: the state read once for scoring, then read and
+    written once by the merge (3 x 553.8 MB), plus the candidates."""
+    B, H, d, n, keep = 64, 16, 64, 192, 128
+    D = d * (d + 1) // 2
+    gen = torch.Generator(device=dev).manual_seed(7)
+    Hst = torch.randn(B, H, D, d, device=dev, generator=gen) * 0.01
+    s = torch.rand(B, H, D, device=dev, generator=gen) + 0.5
+    kc, vc, pos = (x.to(dev) for x in candidate_inputs(B, H, n, d, dtype="bf16", seed=5))
+    state_bytes = float(B * H * D * (d + 1) * 4)
+    nbytes = 3 * state_bytes + float(kc.numel() * 2 * 2 + pos.numel() * 4)
+
+    def step(i):
+        kata.sre_score_topk(Hst, s, kc, vc, pos, keep=keep, merge=True)
+
+    for i in range(max(args.warmup, 2)):
+        step(i)
+    kata.sync_status()
+    barrier(dist_on)
+    iters = max(args.steps // 2, 3)
+    n0 = kata.launch_count()
+    ms = max_over_ranks(time_events(step, iters, stream), dist_on) / iters
+    launches = (kata.launch_count() - n0) // iters
+    kata.sync_status()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    # fp32 work: phi(k)^T [H | s] for every candidate, then a rank-one update
+    # of [H | s] for every merged one (2 flops per multiply-add)
+    flops = float(B * H * (n + (n - keep)) * D * (d + 1) * 2)
+    alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    tflops = flops / (ms / 1e3) / 1e12
+    return {"workload": "sre_b64_h16_d64_n192_keep128", "ms_per_pass": ms, "gbs": gbs,
+            "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_pass": nbytes,
+            "tflops_fp32": tflops, "frac_alu": tflops / alu_peak, "flops_per_pass": flops,
+            "bound": "alu (96 flop per state byte in fp32: SRE decides the kept set, so "
+                     "it stays fp32 on the CUDA cores)",
+            "gpu_launches_per_pass": launches, "l2": "state 554 MB > 126 MB L2"}
 
 
 def bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world):
@@ -499,7 +544,8 @@ def main():
     ap.add_argument("--impl", choices=["kata", "reference"], default="kata")
     ap.add_argument("--headline-only", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode", "long_prefill", "lola"], default=None,
+    ap.add_argument("--only", choices=["decode", "long_prefill", "lola", "sre_stress"],
+                    default=None,
                     help="run one sub-benchmark alone (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -59,6 +59,10 @@ size_t state_partial_smem(int d, int P) {
 }
 
 // part[p][h][i][e] = sum_{r in slice p} phi(x_i)_r H[r][e]; part[..][d] uses s.
+// A CTA loads one slice of H and s once and scores the candidate blocks
+// blockIdx.z, blockIdx.z + gridDim.z, ... against it: with many heads the launch
+// uses gridDim.z = 1 (the state is read once), with few it splits the candidates
+// across CTAs for parallelism.
 template <typename Tin, int DH>
 __global__ void __launch_bounds__(kThreads)
 state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
@@ -66,7 +70,7 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                      float *__restrict__ part) {
     constexpr int D = DH * (DH + 1) / 2;
     constexpr int EQ = DH / 4;
-    const int h = blockIdx.x, p = blockIdx.y, i0 = blockIdx.z * kRows;
+    const int h = blockIdx.x, p = blockIdx.y;
     const int nh = gridDim.x;
     const int slice = (D + P - 1) / P;
     const int r0 = p * slice, r1 = min(D, r0 + slice), nr = max(0, r1 - r0);
@@ -80,40 +84,43 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
 
     build_pair_table(tab, DH);
     const Tin *Xh = X + (size_t)h * x_head_stride;
-    for (int idx = tid; idx < kRows * DH; idx += kThreads) {
-        const int i = idx / DH, a = idx % DH;
-        Xs[i * (DH + 1) + a] = (i0 + i < n) ? to_f32(Xh[(size_t)(i0 + i) * DH + a]) : 0.f;
-    }
     const float4 *H4 = reinterpret_cast<const float4 *>(Hst + ((size_t)h * D + r0) * DH);
     float4 *Hs4 = reinterpret_cast<float4 *>(Hsl);
     for (int idx = tid; idx < nr * DH / 4; idx += kThreads) Hs4[idx] = H4[idx];
     for (int idx = tid; idx < nr; idx += kThreads) ssl[idx] = s[(size_t)h * D + r0 + idx];
-    __syncthreads();
 
     const int i = tid >> 2, eq = (tid & 3) * EQ;
-    const float *xi = Xs + i * (DH + 1);
-    float acc[EQ];
-#pragma unroll
-    for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
-    float den = 0.f;
-    for (int rr = 0; rr < nr; ++rr) {
-        const float ph = phi_entry(xi, tab[r0 + rr]);
-        const float4 *hr = reinterpret_cast<const float4 *>(Hsl + (size_t)rr * DH + eq);
-#pragma unroll
-        for (int c = 0; c < EQ / 4; ++c) {
-            const float4 hv = hr[c];
-            acc[4 * c + 0] = fmaf(ph, hv.x, acc[4 * c + 0]);
-            acc[4 * c + 1] = fmaf(ph, hv.y, acc[4 * c + 1]);
-            acc[4 * c + 2] = fmaf(ph, hv.z, acc[4 * c + 2]);
-            acc[4 * c + 3] = fmaf(ph, hv.w, acc[4 * c + 3]);
+    for (int i0 = blockIdx.z * kRows; i0 < n; i0 += gridDim.z * kRows) {
+        __syncthreads();  // the previous block's reads of Xs are done
+        for (int idx = tid; idx < kRows * DH; idx += kThreads) {
+            const int ii = idx / DH, a = idx % DH;
+            Xs[ii * (DH + 1) + a] = (i0 + ii < n) ? to_f32(Xh[(size_t)(i0 + ii) * DH + a]) : 0.f;
         }
-        den = fmaf(ph, ssl[rr], den);
-    }
-    if (i0 + i < n) {
-        float *dst = part + (((size_t)p * nh + h) * n + i0 + i) * (DH + 1);
+        __syncthreads();
+        const float *xi = Xs + i * (DH + 1);
+        float acc[EQ];
 #pragma unroll
-        for (int c = 0; c < EQ; ++c) dst[eq + c] = acc[c];
-        if (eq == 0) dst[DH] = den;
+        for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
+        float den = 0.f;
+        for (int rr = 0; rr < nr; ++rr) {
+            const float ph = phi_entry(xi, tab[r0 + rr]);
+            const float4 *hr = reinterpret_cast<const float4 *>(Hsl + (size_t)rr * DH + eq);
+#pragma unroll
+            for (int c = 0; c < EQ / 4; ++c) {
+                const float4 hv = hr[c];
+                acc[4 * c + 0] = fmaf(ph, hv.x, acc[4 * c + 0]);
+                acc[4 * c + 1] = fmaf(ph, hv.y, acc[4 * c + 1]);
+                acc[4 * c + 2] = fmaf(ph, hv.z, acc[4 * c + 2]);
+                acc[4 * c + 3] = fmaf(ph, hv.w, acc[4 * c + 3]);
+            }
+            den = fmaf(ph, ssl[rr], den);
+        }
+        if (i0 + i < n) {
+            float *dst = part + (((size_t)p * nh + h) * n + i0 + i) * (DH + 1);
+#pragma unroll
+            for (int c = 0; c < EQ; ++c) dst[eq + c] = acc[c];
+            if (eq == 0) dst[DH] = den;
+        }
     }
 }
 
@@ -122,7 +129,10 @@ cudaError_t launch_state_partial(const Tin *X, long x_head_stride, int nh, int n
                                  const float *Hst, const float *s, int P, float *part,
                                  cudaStream_t stream) {
     const size_t smem = state_partial_smem(d, P);
-    dim3 grid(nh, P, (n + kRows - 1) / kRows);
+    // enough (head, slice) CTAs to fill the GPU twice over: one CTA per slice
+    // reads it once; otherwise split the candidates too
+    const int rb = (n + kRows - 1) / kRows;
+    dim3 grid(nh, P, nh * P >= 2 * kTargetCtas ? 1 : rb);
     cudaError_t err;
 #define KATA_LAUNCH_PARTIAL(DH)                                                               \
     err = cudaFuncSetAttribute(state_partial_kernel<Tin, DH>,                                 \

@@ -227,6 +227,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const long row0 = (long)head * p.nch * kTile;  // first token row of this head
+    // the readout kernel may start its setup and intra-chunk work now; it waits
+    // for this grid's completion before it reads a snapshot
+    if (threadIdx.x == 0) launch_dependents();
 
     if (warp == kTmaWarp) {
         // ---------------- TMA producer ----------------
@@ -624,6 +627,8 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             mbar_arrive_expect_tx(&bar[kRbQFull], kTileBytes);
             tma_load_2d(sm + L::Q, &mq, 0, (int)(row0 + (long)m * kTile), &bar[kRbQFull]);
             load_kv(0);
+            // the snapshots are written by the state kernel just before this one
+            if (n_inter > 0) grid_dependency_wait();
             const int first_p = n_inter < kRP ? n_inter : kRP;
             for (int s = 0; s < first_p; ++s) load_p(s);
             for (int u = 1; u < n_half / 2; ++u) load_kv(u);
@@ -907,7 +912,20 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     auto kern = readout_kernel<DH, NIR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, R::BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(nch, nheads), R::THREADS, R::BYTES, stream>>>(mq, mk, mv, rp);
+    // programmatic dependent launch: overlap this grid's setup and intra-chunk
+    // work with the end of the state kernel
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(nch, nheads, 1);
+    cfg.blockDim = dim3(R::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = R::BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, rp);
+    if (e != cudaSuccess) return e;
     return after_launch();
 }
 
