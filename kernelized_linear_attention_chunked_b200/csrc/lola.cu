@@ -51,75 +51,122 @@ size_t partial_floats(int nh, int n, int d) {
     return (size_t)num_slices(nh, n, d) * nh * n * (d + 1);
 }
 
-size_t state_partial_smem(int d, int P) {
+// Register-blocked scoring: each thread owns kCB candidates x kEB output
+// columns; the state slice streams through shared memory kRC rows at a time
+// and phi of those rows is built once per chunk for all the CTA's candidates.
+constexpr int kRC = 32;  // state rows per chunk
+constexpr int kCB = 4;   // candidates per thread
+constexpr int kEB = 16;  // output columns per thread
+
+// candidates one CTA scores in one pass over its slice
+int partial_pass(int d, int n, int zsplit) {
+    const int neb = d / kEB;
+    const int cap = kThreads / neb * kCB;
+    const int per = (n + zsplit - 1) / zsplit;
+    const int p4 = (per + kCB - 1) / kCB * kCB;
+    return p4 < cap ? p4 : cap;
+}
+
+size_t state_partial_smem(int d, int pass) {
     const int D = packed_dim(d);
-    const int slice = (D + P - 1) / P;
-    return ((size_t)kRows * (d + 1) + (size_t)slice * d + slice) * sizeof(float) +
+    return ((size_t)pass * (d + 1) + (size_t)kRC * pass + (size_t)kRC * d + kRC) * sizeof(float) +
            align_up((size_t)D * sizeof(uint16_t), 16);
 }
 
 // part[p][h][i][e] = sum_{r in slice p} phi(x_i)_r H[r][e]; part[..][d] uses s.
-// A CTA loads one slice of H and s once and scores the candidate blocks
-// blockIdx.z, blockIdx.z + gridDim.z, ... against it: with many heads the launch
-// uses gridDim.z = 1 (the state is read once), with few it splits the candidates
-// across CTAs for parallelism.
+// CTA (h, p, z) scores candidates [z * per, (z + 1) * per) against slice p of
+// head h's state, `pass` candidates at a time; with many heads the launch uses
+// z = 1, so every slice of the state is read once.
 template <typename Tin, int DH>
 __global__ void __launch_bounds__(kThreads)
 state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                      const float *__restrict__ Hst, const float *__restrict__ s, int P,
-                     float *__restrict__ part) {
+                     int pass, float *__restrict__ part) {
     constexpr int D = DH * (DH + 1) / 2;
-    constexpr int EQ = DH / 4;
-    const int h = blockIdx.x, p = blockIdx.y;
-    const int nh = gridDim.x;
+    constexpr int NEB = DH / kEB;  // column blocks
+    const int h = blockIdx.x, p = blockIdx.y, nh = gridDim.x;
     const int slice = (D + P - 1) / P;
-    const int r0 = p * slice, r1 = min(D, r0 + slice), nr = max(0, r1 - r0);
+    const int r0 = p * slice, r1 = min(D, r0 + slice);
+    const int per = (n + gridDim.z - 1) / gridDim.z;
+    const int c0 = blockIdx.z * per, c1 = min(n, c0 + per);
     const int tid = threadIdx.x;
+    const int ej = tid % NEB, cg = tid / NEB;  // column block, candidate group
 
     extern __shared__ float4 smem4[];
-    float *Xs = reinterpret_cast<float *>(smem4);  // [kRows][DH+1]
-    float *Hsl = Xs + kRows * (DH + 1);            // [slice][DH]
-    float *ssl = Hsl + (size_t)slice * DH;         // [slice]
-    uint16_t *tab = reinterpret_cast<uint16_t *>(ssl + slice);
+    float *Xs = reinterpret_cast<float *>(smem4);  // [pass][DH+1]
+    float *Ph = Xs + (size_t)pass * (DH + 1);       // [kRC][pass]
+    float *Hc = Ph + (size_t)kRC * pass;            // [kRC][DH]
+    float *sc = Hc + kRC * DH;                      // [kRC]
+    uint16_t *tab = reinterpret_cast<uint16_t *>(sc + kRC);
 
     build_pair_table(tab, DH);
     const Tin *Xh = X + (size_t)h * x_head_stride;
-    const float4 *H4 = reinterpret_cast<const float4 *>(Hst + ((size_t)h * D + r0) * DH);
-    float4 *Hs4 = reinterpret_cast<float4 *>(Hsl);
-    for (int idx = tid; idx < nr * DH / 4; idx += kThreads) Hs4[idx] = H4[idx];
-    for (int idx = tid; idx < nr; idx += kThreads) ssl[idx] = s[(size_t)h * D + r0 + idx];
+    const float *Hh = Hst + (size_t)h * D * DH;
+    const float *sh = s + (size_t)h * D;
+    const bool active = cg * kCB < pass;
 
-    const int i = tid >> 2, eq = (tid & 3) * EQ;
-    for (int i0 = blockIdx.z * kRows; i0 < n; i0 += gridDim.z * kRows) {
-        __syncthreads();  // the previous block's reads of Xs are done
-        for (int idx = tid; idx < kRows * DH; idx += kThreads) {
-            const int ii = idx / DH, a = idx % DH;
-            Xs[ii * (DH + 1) + a] = (i0 + ii < n) ? to_f32(Xh[(size_t)(i0 + ii) * DH + a]) : 0.f;
+    for (int pc0 = c0; pc0 < c1; pc0 += pass) {
+        const int pn = min(pass, c1 - pc0);
+        __syncthreads();  // the previous pass is done with Xs
+        for (int idx = tid; idx < pass * DH; idx += kThreads) {
+            const int i = idx / DH, a = idx % DH;
+            Xs[i * (DH + 1) + a] = i < pn ? to_f32(Xh[(size_t)(pc0 + i) * DH + a]) : 0.f;
         }
-        __syncthreads();
-        const float *xi = Xs + i * (DH + 1);
-        float acc[EQ];
+        float acc[kCB][kEB];
+        float den[kCB];
 #pragma unroll
-        for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
-        float den = 0.f;
-        for (int rr = 0; rr < nr; ++rr) {
-            const float ph = phi_entry(xi, tab[r0 + rr]);
-            const float4 *hr = reinterpret_cast<const float4 *>(Hsl + (size_t)rr * DH + eq);
+        for (int c = 0; c < kCB; ++c) {
+            den[c] = 0.f;
 #pragma unroll
-            for (int c = 0; c < EQ / 4; ++c) {
-                const float4 hv = hr[c];
-                acc[4 * c + 0] = fmaf(ph, hv.x, acc[4 * c + 0]);
-                acc[4 * c + 1] = fmaf(ph, hv.y, acc[4 * c + 1]);
-                acc[4 * c + 2] = fmaf(ph, hv.z, acc[4 * c + 2]);
-                acc[4 * c + 3] = fmaf(ph, hv.w, acc[4 * c + 3]);
+            for (int e = 0; e < kEB; ++e) acc[c][e] = 0.f;
+        }
+        for (int rc = r0; rc < r1; rc += kRC) {
+            const int nr = min(kRC, r1 - rc);
+            __syncthreads();  // Xs written; the previous chunk's readers are done
+            for (int idx = tid; idx < nr * DH / 4; idx += kThreads)
+                reinterpret_cast<float4 *>(Hc)[idx] =
+                    reinterpret_cast<const float4 *>(Hh + (size_t)rc * DH)[idx];
+            for (int idx = tid; idx < nr; idx += kThreads) sc[idx] = sh[rc + idx];
+            for (int idx = tid; idx < nr * pass; idx += kThreads) {
+                const int rr = idx / pass, i = idx % pass;
+                Ph[rr * pass + i] = phi_entry(Xs + i * (DH + 1), tab[rc + rr]);
             }
-            den = fmaf(ph, ssl[rr], den);
-        }
-        if (i0 + i < n) {
-            float *dst = part + (((size_t)p * nh + h) * n + i0 + i) * (DH + 1);
+            __syncthreads();
+            if (active) {
+                for (int rr = 0; rr < nr; ++rr) {
+                    const float4 ph = *reinterpret_cast<const float4 *>(Ph + rr * pass + cg * kCB);
+                    const float pv[kCB] = {ph.x, ph.y, ph.z, ph.w};
+                    const float4 *hv = reinterpret_cast<const float4 *>(Hc + rr * DH + ej * kEB);
 #pragma unroll
-            for (int c = 0; c < EQ; ++c) dst[eq + c] = acc[c];
-            if (eq == 0) dst[DH] = den;
+                    for (int q = 0; q < kEB / 4; ++q) {
+                        const float4 hq = hv[q];
+#pragma unroll
+                        for (int c = 0; c < kCB; ++c) {
+                            acc[c][4 * q + 0] = fmaf(pv[c], hq.x, acc[c][4 * q + 0]);
+                            acc[c][4 * q + 1] = fmaf(pv[c], hq.y, acc[c][4 * q + 1]);
+                            acc[c][4 * q + 2] = fmaf(pv[c], hq.z, acc[c][4 * q + 2]);
+                            acc[c][4 * q + 3] = fmaf(pv[c], hq.w, acc[c][4 * q + 3]);
+                        }
+                    }
+                    if (ej == 0) {
+                        const float sr = sc[rr];
+#pragma unroll
+                        for (int c = 0; c < kCB; ++c) den[c] = fmaf(pv[c], sr, den[c]);
+                    }
+                }
+            }
+        }
+        if (active) {
+#pragma unroll
+            for (int c = 0; c < kCB; ++c) {
+                const int i = pc0 + cg * kCB + c;
+                if (i < c1) {
+                    float *dst = part + (((size_t)p * nh + h) * n + i) * (DH + 1);
+#pragma unroll
+                    for (int e = 0; e < kEB; ++e) dst[ej * kEB + e] = acc[c][e];
+                    if (ej == 0) dst[DH] = den[c];
+                }
+            }
         }
     }
 }
@@ -128,18 +175,20 @@ template <typename Tin>
 cudaError_t launch_state_partial(const Tin *X, long x_head_stride, int nh, int n, int d,
                                  const float *Hst, const float *s, int P, float *part,
                                  cudaStream_t stream) {
-    const size_t smem = state_partial_smem(d, P);
     // enough (head, slice) CTAs to fill the GPU twice over: one CTA per slice
     // reads it once; otherwise split the candidates too
     const int rb = (n + kRows - 1) / kRows;
-    dim3 grid(nh, P, nh * P >= 2 * kTargetCtas ? 1 : rb);
+    const int zsplit = nh * P >= 2 * kTargetCtas ? 1 : rb;
+    const int pass = partial_pass(d, n, zsplit);
+    const size_t smem = state_partial_smem(d, pass);
+    dim3 grid(nh, P, zsplit);
     cudaError_t err;
 #define KATA_LAUNCH_PARTIAL(DH)                                                               \
     err = cudaFuncSetAttribute(state_partial_kernel<Tin, DH>,                                 \
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);      \
     if (err != cudaSuccess) return err;                                                       \
     state_partial_kernel<Tin, DH><<<grid, kThreads, smem, stream>>>(X, x_head_stride, n, Hst, \
-                                                                     s, P, part);
+                                                                     s, P, pass, part);
     switch (d) {
         case 16: KATA_LAUNCH_PARTIAL(16) break;
         case 32: KATA_LAUNCH_PARTIAL(32) break;
