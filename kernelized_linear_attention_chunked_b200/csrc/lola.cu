@@ -220,20 +220,33 @@ sre_select_kernel(const float *__restrict__ part, int P, int n, int d,
     __shared__ unsigned char kept[1024];
     const int h = blockIdx.x, nh = gridDim.x, j = threadIdx.x;
     const int m = keep < n ? keep : n;
-    if (j < n) {
-        float den = 0.f;
-        for (int p = 0; p < P; ++p) den += part[(((size_t)p * nh + h) * n + j) * (d + 1) + d];
-        const float inv = 1.f / (den + eps);
-        const Tin *vj = vc + (size_t)h * cand_head_stride + (size_t)j * d;
-        float err = 0.f;
-        for (int e = 0; e < d; ++e) {
-            float num = 0.f;
-            for (int p = 0; p < P; ++p) num += part[(((size_t)p * nh + h) * n + j) * (d + 1) + e];
-            const float diff = num * inv - to_f32(vj[e]);
-            err = fmaf(diff, diff, err);
+    // SRE of every candidate: one warp per candidate, lanes across the columns
+    // of its partial sums (coalesced), summed over the slices in slice order
+    {
+        const int warp = j >> 5, lane = j & 31, nwarps = blockDim.x >> 5;
+        const size_t pstride = (size_t)nh * n * (d + 1);
+        for (int c = warp; c < n; c += nwarps) {
+            const float *pc = part + ((size_t)h * n + c) * (d + 1);
+            float den = 0.f;
+            if (lane == 0)
+                for (int p = 0; p < P; ++p) den += pc[p * pstride + d];
+            den = __shfl_sync(0xFFFFFFFFu, den, 0);
+            const float inv = 1.f / (den + eps);
+            const Tin *vj = vc + (size_t)h * cand_head_stride + (size_t)c * d;
+            float err = 0.f;
+            for (int e = lane; e < d; e += 32) {
+                float num = 0.f;
+                for (int p = 0; p < P; ++p) num += pc[p * pstride + e];
+                const float diff = num * inv - to_f32(vj[e]);
+                err = fmaf(diff, diff, err);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xFFFFFFFFu, err, o);
+            if (lane == 0) {
+                sc[c] = isnan(err) ? -INFINITY : err;  // a total order even for 0/0 scores
+                ps[c] = pos[(size_t)h * pos_head_stride + c];
+            }
         }
-        sc[j] = isnan(err) ? -INFINITY : err;  // a total order even for 0/0 scores
-        ps[j] = pos[(size_t)h * pos_head_stride + j];
     }
     __syncthreads();
     bool isk = false;
@@ -260,56 +273,101 @@ sre_select_kernel(const float *__restrict__ part, int P, int n, int d,
     if (j == 0) mcount[h] = n - m;
 }
 
+// Merge: Hdst[r][e] = Hsrc[r][e] + sum_{c merged} phi(k_c)_r v_c[e], and the
+// same for s. CTA (h, 256-row block); thread = 4 rows x 16 columns of the
+// block, accumulating over the merged candidates kMC at a time (phi of the
+// block's rows built once per chunk in shared memory); the state is read and
+// written once with 16-byte accesses. Hdst may alias Hsrc.
+constexpr int kMR = 256;  // state rows per CTA
+constexpr int kMC = 16;   // merged candidates per shared-memory chunk
+
 template <typename Tin, int DH>
 __global__ void __launch_bounds__(kThreads)
 merge_kernel(const float *Hsrc, const float *ssrc, float *Hdst, float *sdst,
              const Tin *__restrict__ kc, const Tin *__restrict__ vc, long cand_head_stride,
-             const int *__restrict__ mlist, const int *__restrict__ mcount, int n, int P) {
+             const int *__restrict__ mlist, const int *__restrict__ mcount, int n) {
     constexpr int D = DH * (DH + 1) / 2;
-    constexpr int EQ = DH / 4;
-    __shared__ float Ks[kRows][DH + 1];
-    __shared__ float Vs[kRows][DH];
+    constexpr int NEB = DH / kEB;  // column blocks
+    __shared__ float Ks[kMC][DH + 1];
+    __shared__ __align__(16) float Vs[kMC][DH];
+    __shared__ __align__(16) float Pk[kMC][kMR];
     __shared__ uint16_t tab[D];
-    const int h = blockIdx.x, p = blockIdx.y, tid = threadIdx.x;
-    const int slice = (D + P - 1) / P;
-    const int r0 = p * slice, r1 = min(D, r0 + slice);
+    const int h = blockIdx.x, rb0 = blockIdx.y * kMR, tid = threadIdx.x;
     const int m = mcount[h];
+    const bool active = tid < (kMR / 4) * NEB;
+    const int rg = tid / NEB, ej = tid % NEB;
     build_pair_table(tab, DH);
     const Tin *kh = kc + (size_t)h * cand_head_stride;
     const Tin *vh = vc + (size_t)h * cand_head_stride;
-    const int eq = (tid & 3) * EQ;
-    for (int rb = r0; rb < r1; rb += kRows) {
-        const int r = rb + (tid >> 2);
-        float acc[EQ];
+    float acc[4][kEB];
+    float sacc[4];
 #pragma unroll
-        for (int c = 0; c < EQ; ++c) acc[c] = 0.f;
-        float sacc = 0.f;
-        for (int mb = 0; mb < m; mb += kRows) {
-            const int nb = min(kRows, m - mb);
-            __syncthreads();
-            for (int idx = tid; idx < nb * DH; idx += kThreads) {
-                const int ii = idx / DH, a = idx % DH;
-                const int j = mlist[(size_t)h * n + mb + ii];
-                Ks[ii][a] = to_f32(kh[(size_t)j * DH + a]);
-                Vs[ii][a] = to_f32(vh[(size_t)j * DH + a]);
+    for (int r = 0; r < 4; ++r) {
+        sacc[r] = 0.f;
+#pragma unroll
+        for (int e = 0; e < kEB; ++e) acc[r][e] = 0.f;
+    }
+    for (int mc = 0; mc < m; mc += kMC) {
+        const int nb = min(kMC, m - mc);
+        __syncthreads();  // the previous chunk's readers are done
+        for (int idx = tid; idx < kMC * DH; idx += kThreads) {
+            const int ii = idx / DH, a = idx % DH;
+            float kx = 0.f, vx = 0.f;
+            if (ii < nb) {
+                const int j = mlist[(size_t)h * n + mc + ii];
+                kx = to_f32(kh[(size_t)j * DH + a]);
+                vx = to_f32(vh[(size_t)j * DH + a]);
             }
-            __syncthreads();
-            if (r < r1) {
-                const uint16_t ab = tab[r];
-                for (int ii = 0; ii < nb; ++ii) {
-                    const float pk = phi_entry(Ks[ii], ab);
-                    sacc += pk;
+            Ks[ii][a] = kx;
+            Vs[ii][a] = vx;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kMC * kMR; idx += kThreads) {
+            const int ii = idx / kMR, rr = idx % kMR;
+            Pk[ii][rr] = rb0 + rr < D ? phi_entry(Ks[ii], tab[rb0 + rr]) : 0.f;
+        }
+        __syncthreads();
+        if (active) {
+            for (int ii = 0; ii < nb; ++ii) {
+                const float4 p4 = *reinterpret_cast<const float4 *>(&Pk[ii][rg * 4]);
+                const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
+                const float4 *vv = reinterpret_cast<const float4 *>(&Vs[ii][ej * kEB]);
 #pragma unroll
-                    for (int c = 0; c < EQ; ++c) acc[c] = fmaf(pk, Vs[ii][eq + c], acc[c]);
+                for (int q = 0; q < kEB / 4; ++q) {
+                    const float4 vq = vv[q];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        acc[r][4 * q + 0] = fmaf(pr[r], vq.x, acc[r][4 * q + 0]);
+                        acc[r][4 * q + 1] = fmaf(pr[r], vq.y, acc[r][4 * q + 1]);
+                        acc[r][4 * q + 2] = fmaf(pr[r], vq.z, acc[r][4 * q + 2]);
+                        acc[r][4 * q + 3] = fmaf(pr[r], vq.w, acc[r][4 * q + 3]);
+                    }
+                }
+                if (ej == 0) {
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) sacc[r] += pr[r];
                 }
             }
         }
-        if (r < r1) {
-            const size_t base = ((size_t)h * D + r) * DH + eq;
+    }
+    if (!active) return;
 #pragma unroll
-            for (int c = 0; c < EQ; ++c) Hdst[base + c] = Hsrc[base + c] + acc[c];
-            if (eq == 0) sdst[(size_t)h * D + r] = ssrc[(size_t)h * D + r] + sacc;
+    for (int r = 0; r < 4; ++r) {
+        const int row = rb0 + rg * 4 + r;
+        if (row >= D) break;
+        const size_t base = ((size_t)h * D + row) * DH + ej * kEB;
+        const float4 *src = reinterpret_cast<const float4 *>(Hsrc + base);
+        float4 *dst = reinterpret_cast<float4 *>(Hdst + base);
+#pragma unroll
+        for (int q = 0; q < kEB / 4; ++q) {
+            float4 x = src[q];
+            x.x += acc[r][4 * q + 0];
+            x.y += acc[r][4 * q + 1];
+            x.z += acc[r][4 * q + 2];
+            x.w += acc[r][4 * q + 3];
+            dst[q] = x;
         }
+        if (ej == 0) sdst[(size_t)h * D + row] = ssrc[(size_t)h * D + row] + sacc[r];
     }
 }
 
@@ -460,12 +518,11 @@ cudaError_t sre_impl(const float *Hst, const float *s, const Tin *kc, const Tin 
         return cudaSuccess;
     }
     const int D = packed_dim(d);
-    const int P2 = (D + 127) / 128;
-    dim3 grid(nh, P2);
+    dim3 grid(nh, (D + kMR - 1) / kMR);
     switch (d) {
-        case 16: merge_kernel<Tin, 16><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
-        case 32: merge_kernel<Tin, 32><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
-        case 64: merge_kernel<Tin, 64><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n, P2); break;
+        case 16: merge_kernel<Tin, 16><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n); break;
+        case 32: merge_kernel<Tin, 32><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n); break;
+        case 64: merge_kernel<Tin, 64><<<grid, kThreads, 0, stream>>>(Hst, s, Hst_mut, s_mut, kc, vc, cstride, w.mlist, w.mcount, n); break;
         default: return cudaErrorInvalidValue;
     }
     return after_launch();
