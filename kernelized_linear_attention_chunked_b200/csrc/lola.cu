@@ -228,14 +228,17 @@ sre_select_kernel(const float *__restrict__ part, int P, int n, int d,
         for (int c = warp; c < n; c += nwarps) {
             const float *pc = part + ((size_t)h * n + c) * (d + 1);
             float den = 0.f;
-            if (lane == 0)
+            if (lane == 0) {
+#pragma unroll 4
                 for (int p = 0; p < P; ++p) den += pc[p * pstride + d];
+            }
             den = __shfl_sync(0xFFFFFFFFu, den, 0);
             const float inv = 1.f / (den + eps);
             const Tin *vj = vc + (size_t)h * cand_head_stride + (size_t)c * d;
             float err = 0.f;
             for (int e = lane; e < d; e += 32) {
                 float num = 0.f;
+#pragma unroll 4
                 for (int p = 0; p < P; ++p) num += pc[p * pstride + e];
                 const float diff = num * inv - to_f32(vj[e]);
                 err = fmaf(diff, diff, err);
@@ -500,7 +503,9 @@ cudaError_t sre_impl(const float *Hst, const float *s, const Tin *kc, const Tin 
     const long cstride = (long)cand_stride * d;
     cudaError_t err = launch_state_partial<Tin>(kc, cstride, nh, n, d, Hst, s, P, w.part, stream);
     if (err != cudaSuccess) return err;
-    const int threads = ((n + 31) / 32) * 32;
+    // 32 warps share the per-candidate reductions; the ranking uses one thread
+    // per candidate (n <= 1024)
+    const int threads = 1024;
     sre_select_kernel<Tin><<<nh, threads, 0, stream>>>(w.part, P, n, d, vc, cstride, pos,
                                                        cand_stride, keep, eps, scores, keep_idx,
                                                        w.mlist, w.mcount);
