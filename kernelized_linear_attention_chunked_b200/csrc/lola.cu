@@ -136,10 +136,12 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                 for (int rr = 0; rr < nr; ++rr) {
                     const float4 ph = *reinterpret_cast<const float4 *>(Ph + rr * pass + cg * kCB);
                     const float pv[kCB] = {ph.x, ph.y, ph.z, ph.w};
-                    const float4 *hv = reinterpret_cast<const float4 *>(Hc + rr * DH + ej * kEB);
+                    // columns 4 (q NEB + ej) .. +3: neighbouring threads read
+                    // neighbouring 16-byte chunks (no bank conflicts)
+                    const float4 *hv = reinterpret_cast<const float4 *>(Hc + rr * DH);
 #pragma unroll
                     for (int q = 0; q < kEB / 4; ++q) {
-                        const float4 hq = hv[q];
+                        const float4 hq = hv[q * NEB + ej];
 #pragma unroll
                         for (int c = 0; c < kCB; ++c) {
                             acc[c][4 * q + 0] = fmaf(pv[c], hq.x, acc[c][4 * q + 0]);
@@ -163,7 +165,9 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                 if (i < c1) {
                     float *dst = part + (((size_t)p * nh + h) * n + i) * (DH + 1);
 #pragma unroll
-                    for (int e = 0; e < kEB; ++e) dst[ej * kEB + e] = acc[c][e];
+                    for (int q = 0; q < kEB / 4; ++q)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) dst[4 * (q * NEB + ej) + k] = acc[c][4 * q + k];
                     if (ej == 0) dst[DH] = den[c];
                 }
             }
@@ -334,10 +338,11 @@ merge_kernel(const float *Hsrc, const float *ssrc, float *Hdst, float *sdst,
             for (int ii = 0; ii < nb; ++ii) {
                 const float4 p4 = *reinterpret_cast<const float4 *>(&Pk[ii][rg * 4]);
                 const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
-                const float4 *vv = reinterpret_cast<const float4 *>(&Vs[ii][ej * kEB]);
+                // columns 4 (q NEB + ej) .. +3 (neighbouring threads, neighbouring chunks)
+                const float4 *vv = reinterpret_cast<const float4 *>(&Vs[ii][0]);
 #pragma unroll
                 for (int q = 0; q < kEB / 4; ++q) {
-                    const float4 vq = vv[q];
+                    const float4 vq = vv[q * NEB + ej];
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         acc[r][4 * q + 0] = fmaf(pr[r], vq.x, acc[r][4 * q + 0]);
@@ -358,17 +363,17 @@ merge_kernel(const float *Hsrc, const float *ssrc, float *Hdst, float *sdst,
     for (int r = 0; r < 4; ++r) {
         const int row = rb0 + rg * 4 + r;
         if (row >= D) break;
-        const size_t base = ((size_t)h * D + row) * DH + ej * kEB;
+        const size_t base = ((size_t)h * D + row) * DH;
         const float4 *src = reinterpret_cast<const float4 *>(Hsrc + base);
         float4 *dst = reinterpret_cast<float4 *>(Hdst + base);
 #pragma unroll
         for (int q = 0; q < kEB / 4; ++q) {
-            float4 x = src[q];
+            float4 x = src[q * NEB + ej];
             x.x += acc[r][4 * q + 0];
             x.y += acc[r][4 * q + 1];
             x.z += acc[r][4 * q + 2];
             x.w += acc[r][4 * q + 3];
-            dst[q] = x;
+            dst[q * NEB + ej] = x;
         }
         if (ej == 0) sdst[(size_t)h * D + row] = ssrc[(size_t)h * D + row] + sacc[r];
     }
