@@ -42,6 +42,28 @@ def test_sre_topk_merge(dtype, d, n, keep):
     assert rel_l2(Hg, Hr) < 1e-5 and rel_l2(sg, sr) < 1e-5
 
 
+@pytest.mark.parametrize("d", [32, 64])
+def test_sre_topk_merge_many_heads(d):
+    # 320 heads: enough (head, slice) pairs that one CTA scores every candidate
+    # against its slice of the state (the state is read once)
+    B, H, n, keep = 8, 40, 130, 64
+    H0, s0 = oracle_state(B, H, d, 100, seed=d + 1)
+    kc, vc, pos = candidate_inputs(B, H, n, d, dtype="bf16", seed=n + d)
+    Hg, sg = cuda(H0.clone(), s0.clone())
+    sc, ki = kata.sre_score_topk(Hg, sg, *cuda(kc, vc, pos), keep=keep, eps=1e-6, merge=True)
+    kata.sync_status()
+    rsc = oracle.sre(H0, s0, kc, vc, 1e-6)
+    assert rel_l2(sc, rsc) < REL_F32
+    rki = oracle.topk(rsc, pos.numpy(), keep)
+    ki = ki.cpu().numpy()
+    for b in range(B):
+        for h in range(H):
+            assert allowed_swap(rsc[b, h], ki[b, h], rki[b, h], keep)
+    Hr, sr = H0.double().numpy().copy(), s0.double().numpy().copy()
+    oracle.merge(Hr, sr, kc, vc, ki)
+    assert rel_l2(Hg, Hr) < 1e-5 and rel_l2(sg, sr) < 1e-5
+
+
 def test_sre_ties_go_to_smaller_position():
     B, H, n, d = 1, 2, 40, 32
     H0, s0 = oracle_state(B, H, d, 100, seed=1)
