@@ -1,9 +1,11 @@
 """Benchmark of causal kernelized linear attention (phi(x) = x x^T) on B200.
 
-Headline (``value``): chunked-prefill tokens/s on the prefill workload
-B=4, H=8, T=2048, d=32, bf16, chunk 64 -- one step is one kata_prefill call
-over that batch (feature map, intra-chunk contraction, state accumulation,
-carry and readout). The same JSON line carries the decode step (B=64, H=16,
+Headline (``value``): prefill tokens/s on the prefill workload B=4, H=8,
+T=2048, d=32, bf16, chunk 64 -- one step is one output-only kata_prefill call
+over that batch. For this size kata_prefill takes the quadratic form (one
+tcgen05 kernel, (Q K^T)^2 [V | 1]); the same call in the chunked form (state
+accumulation and carry, then the readout) is timed beside it under
+``chunked_form``. The same JSON line carries the decode step (B=64, H=16,
 d=64 from a 4096-token prefix), the long prefill (B=2, H=16, T=16384, d=64)
 and the LoLA schedule (B=2, H=8, T=8192, d=64) as sub-results, the roofline
 of the dominant kernel, the fp64 oracle timed on the host cores, and an
@@ -50,6 +52,12 @@ def prefill_flops(w) -> float:
     D = w.d * (w.d + 1) // 2
     per = 4 * D * (w.d + 1) + (w.chunk + 1) * (2 * w.d + 1)
     return float(per) * w.B * w.H * w.T
+
+
+def quadratic_flops(w) -> float:
+    """Algorithmic flops of the quadratic form: per causal pair (j <= i) 2d for
+    q.k, 2d for the weighted v and 2 for the denominator."""
+    return float(w.T * (w.T + 1) // 2 * (4 * w.d + 2)) * w.B * w.H
 
 
 def prefill_update_flops(w) -> float:
@@ -306,57 +314,39 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     tokens_per_step = w.B * w.T
     value = world * tokens_per_step * args.steps / (ms / 1e3)
     ms_step = ms / args.steps
-    flops = prefill_flops(w)
-    tflops = flops / (ms_step / 1e3) / 1e12
-
-    # roofline of the dominant kernel. The tensor-core path is two launches per
-    # call: the state kernel (chunk-state accumulation and carry, half the
-    # inter-chunk flops) and the readout kernel (the other half plus the
-    # intra-chunk part). The state kernel is timed alone by a state-only call
-    # (it then writes the final state instead of the snapshots); the readout is
-    # the difference.
-    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    # the form kata_prefill takes for this output-only call, and its flops
+    form = kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16, True)
     path = "tc" if kata.prefill_uses_tensor_cores(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16) \
         else "simt"
-    kernels = None
-    if path == "tc":
-        Hs = torch.empty(w.B, w.H, w.D, w.d, device=dev)
-        ss = torch.empty(w.B, w.H, w.D, device=dev)
-
-        def state_step(i):
-            qq, kk, vv = sets[i % R]
-            kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, output=False, H_out=Hs,
-                         s_out=ss, workspace=ws)
-
-        for i in range(3):
-            state_step(i)
-        lat_state = per_launch_ms(state_step, max(args.steps, 5), stream)
-        lat_read = max(lat - lat_state, 1e-6)
-        f_update = prefill_update_flops(w)
-        f_read = flops - f_update
-        kernels = {
-            "state_kernel": {"ms": lat_state, "tflops": f_update / (lat_state / 1e3) / 1e12},
-            "readout_kernel": {"ms": lat_read, "tflops": f_read / (lat_read / 1e3) / 1e12,
-                               "note": "call time minus the state-only call"}}
-        dom = "state_kernel" if lat_state >= lat_read else "readout_kernel"
-        dom_ms = lat_state if dom == "state_kernel" else lat_read
-        dom_flops = f_update if dom == "state_kernel" else f_read
-        roof = {"bound": "tensor", "achieved": dom_flops / (dom_ms / 1e3) / 1e12,
+    flops = quadratic_flops(w) if form == "quadratic" else prefill_flops(w)
+    tflops = flops / (ms_step / 1e3) / 1e12
+    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    chunked = None
+    if form == "quadratic":
+        # one launch per call: the quadratic-form kernel
+        roof = {"bound": "tensor", "achieved": flops / (lat / 1e3) / 1e12,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        kernel = dom
-        del Hs, ss
+        kernel, dom_ms, kernels = "quad_kernel", lat, None
+        chunked = bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks)
+    elif path == "tc":
+        kernels = chunked_kernels(kata, w, sets, R, ws, args, stream, dev, lat)
+        dom = max(kernels, key=lambda n: kernels[n]["ms"])
+        roof = {"bound": "tensor", "achieved": kernels[dom]["tflops"],
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        kernel, dom_ms = dom, kernels[dom]["ms"]
     else:
         # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x max SM clock
         alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof = {"bound": "alu", "achieved": flops / (lat / 1e3) / 1e12, "peak": alu_peak,
                 "unit": "TFLOP/s"}
-        kernel = "prefill_simt_kernel"
-        dom_ms = lat
+        kernel, dom_ms, kernels = "prefill_simt_kernel", lat, None
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
         else "fallback"
     roof["kernel"] = kernel
     roof["launch_ms"] = dom_ms
+    roof["algorithmic_flops"] = flops if kernel in ("quad_kernel", "prefill_simt_kernel") \
+        else None
     roof["traffic"] = traffic_record(kernel, HEADLINE)
     roof["call_ms"] = lat
     roof["call_tflops"] = flops / (lat / 1e3) / 1e12
@@ -397,15 +387,68 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
             "data": "synthetic",
             "config": {"workload": HEADLINE, "global_batch": w.B * world, "seq_len": w.T,
                        "heads": w.H, "head_dim": w.d, "packed_dim": w.D, "chunk": w.chunk,
-                       "parallelism": f"dp{world}", "path": path,
+                       "parallelism": f"dp{world}", "path": path, "form": form,
                        "l2": f"{R} rotating input sets ({R * prefill_bytes(w) / 2**20:.0f} MB "
                              "> 126 MB L2)"},
-            "prefill": {"tflops": tflops, "frac_bf16_peak": tflops / peaks["bf16_tflops"],
+            "prefill": {"form": form, "flops_per_step": flops, "tflops": tflops,
+                        "frac_bf16_peak": tflops / peaks["bf16_tflops"],
                         "peak_source": peak_kind},
+            "chunked_form": chunked,
             "roofline": roof, "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches,
             "wall_s": wall}
     line.update(sub)
     return line
+
+
+def chunked_kernels(kata, w, sets, R, ws, args, stream, dev, lat_call):
+    """Per-kernel times of the chunked form's two launches: the state kernel
+    (chunk-state accumulation and carry, half the inter-chunk flops) timed alone
+    by a state-only call (it then writes the final state instead of the
+    snapshots), and the readout kernel (the other half plus the intra-chunk
+    part) as the call time minus that."""
+    flops = prefill_flops(w)
+    Hs = torch.empty(w.B, w.H, w.D, w.d, device=dev)
+    ss = torch.empty(w.B, w.H, w.D, device=dev)
+
+    def state_step(i):
+        qq, kk, vv = sets[i % R]
+        kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, output=False, H_out=Hs, s_out=ss,
+                     workspace=ws, form="chunked")
+
+    for i in range(3):
+        state_step(i)
+    lat_state = per_launch_ms(state_step, max(args.steps, 5), stream)
+    lat_read = max(lat_call - lat_state, 1e-6)
+    f_update = prefill_update_flops(w)
+    f_read = flops - f_update
+    return {"state_kernel": {"ms": lat_state, "tflops": f_update / (lat_state / 1e3) / 1e12,
+                             "traffic": traffic_record("state_kernel", HEADLINE)},
+            "readout_kernel": {"ms": lat_read, "tflops": f_read / (lat_read / 1e3) / 1e12,
+                               "traffic": traffic_record("readout_kernel", HEADLINE),
+                               "note": "call time minus the state-only call"}}
+
+
+def bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks):
+    """The same output-only call in the chunked form (state kernel + readout
+    kernel), for comparison with the quadratic form that kata_prefill takes."""
+    outs = [torch.empty(w.B, w.H, w.T, w.d, device=dev) for _ in range(R)]
+
+    def step(i):
+        qq, kk, vv = sets[i % R]
+        kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, state=False, o=outs[i % R],
+                     workspace=ws, form="chunked")
+
+    for i in range(args.warmup):
+        step(i)
+    ms = time_events(step, args.steps, stream) / args.steps
+    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    kata.sync_status()
+    flops = prefill_flops(w)
+    return {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+            "flops_per_step": flops, "tflops": flops / (ms / 1e3) / 1e12,
+            "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "call_ms": lat,
+            "kernels": chunked_kernels(kata, w, sets, R, ws, args, stream, dev, lat)}
 
 
 def bench_decode(kata, args, dev, stream, peaks, dist_on, world):

@@ -109,14 +109,50 @@ KATA_API size_t kata_prefill_workspace_bytes(int B, int H, int T, int d, int chu
  *   workspace device scratch of at least kata_prefill_workspace_bytes().
  * bf16 inputs run on the tcgen05 tensor cores (bf16 operands, fp32
  * accumulation and state); fp32 inputs run in fp32 on the CUDA cores.
+ * An output-only bf16 call (no H_in, no H_out) with T up to
+ * kata_quadratic_max_tokens(d) runs the quadratic form instead (see
+ * kata_prefill_ex); the result is the same up to rounding.
  */
 KATA_API int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
                  int d, int chunk, float eps, const float *H_in, const float *s_in, float *o,
                  float *H_out, float *s_out, void *workspace, size_t ws_bytes, void *stream);
 
-/* Which kernel kata_prefill runs for these sizes: 1 = tcgen05 tensor cores,
- * 0 = CUDA cores, -1 = invalid or unsupported arguments. */
+/* Which kernel the chunked form runs for these sizes: 1 = tcgen05 tensor
+ * cores, 0 = CUDA cores, -1 = invalid or unsupported arguments. */
 KATA_API int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype);
+
+/* The two exact forms of a prefill. */
+enum { KATA_FORM_AUTO = 0, KATA_FORM_CHUNKED = 1, KATA_FORM_QUADRATIC = 2 };
+
+/*
+ * kata_prefill with the form chosen by the caller.
+ *   KATA_FORM_CHUNKED    the chunked state form described at kata_prefill.
+ *   KATA_FORM_QUADRATIC  the quadratic form [KATA s2.2: the rank-one PSD
+ *                        feature makes the kernel (q.k)^2]:
+ *                          o_i = sum_{j<=i} (q_i.k_j)^2 v_j / (sum_{j<=i} (q_i.k_j)^2 + eps),
+ *                        O(T^2 d) work on the tcgen05 tensor cores with no
+ *                        state (bf16 (q.k)^2 operands, fp32 accumulation). It
+ *                        takes bf16 inputs, d = 32 or 64, T a multiple of 128,
+ *                        o non-NULL and H_in, s_in, H_out, s_out NULL; other
+ *                        calls return KATA_ERR_UNSUPPORTED. workspace is not
+ *                        used (may be NULL, ws_bytes 0).
+ *   KATA_FORM_AUTO       what kata_prefill does: the quadratic form when it
+ *                        applies and T <= kata_quadratic_max_tokens(d), the
+ *                        chunked form otherwise.
+ * Both forms give the same result up to rounding.
+ */
+KATA_API int kata_prefill_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                    int T, int d, int chunk, float eps, const float *H_in, const float *s_in,
+                    float *o, float *H_out, float *s_out, void *workspace, size_t ws_bytes,
+                    void *stream, int form);
+
+/* Largest T for which KATA_FORM_AUTO takes the quadratic form (0: never). */
+KATA_API int kata_quadratic_max_tokens(int d);
+
+/* The form KATA_FORM_AUTO takes for these sizes: KATA_FORM_CHUNKED or
+ * KATA_FORM_QUADRATIC; output_only = o given, no initial or final state.
+ * -1 = invalid or unsupported arguments. */
+KATA_API int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int output_only);
 
 /* Device workspace for kata_prefill_host: staging for q, k, v and o plus
  * kata_prefill_workspace_bytes(). */

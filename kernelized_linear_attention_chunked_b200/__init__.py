@@ -7,6 +7,7 @@ its thin Python binding plus the seeded synthetic input generators.
 from ._binding import (  # noqa: F401
     KATA_BF16,
     KATA_F32,
+    FORMS,
     LIB_PATH,
     SIGNATURES,
     KataError,
@@ -19,10 +20,12 @@ from ._binding import (  # noqa: F401
     lola_prefill_workspace_bytes,
     packed_dim,
     prefill,
+    prefill_auto_form,
     prefill_host,
     prefill_host_workspace_bytes,
     prefill_uses_tensor_cores,
     prefill_workspace_bytes,
+    quadratic_max_tokens,
     sre_score_topk,
     sync_status,
 )

@@ -32,6 +32,10 @@ SIGNATURES = {
     "kata_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
                           _vp, _sz, _vp]),
     "kata_prefill_path": (_i, [_i, _i, _i, _i, _i, _i]),
+    "kata_prefill_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
+                             _vp, _sz, _vp, _i]),
+    "kata_quadratic_max_tokens": (_i, [_i]),
+    "kata_prefill_auto_form": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "kata_prefill_host_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "kata_prefill_host": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "kata_decode_step": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp]),
@@ -119,10 +123,16 @@ def sync_status(stream=None) -> None:
     _check("kata_sync_status", lib().kata_sync_status(_stream(stream)))
 
 
+# kata_prefill_ex forms
+FORMS = {"auto": 0, "chunked": 1, "quadratic": 2}
+
+
 def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state: bool = True,
-            output: bool = True, o=None, H_out=None, s_out=None, workspace=None, stream=None):
-    """Causal chunked prefill. q, k, v [B, H, T, d]. Returns (o, H, s); o is None
-    when ``output`` is False (state only), H and s are None when ``state`` is False."""
+            output: bool = True, o=None, H_out=None, s_out=None, workspace=None, stream=None,
+            form: str = "auto"):
+    """Causal prefill. q, k, v [B, H, T, d]. Returns (o, H, s); o is None when
+    ``output`` is False (state only), H and s are None when ``state`` is False.
+    ``form``: "chunked", "quadratic" (output only) or "auto" (kata_prefill's choice)."""
     _dev(q, k, v, H_in, s_in)
     B, Hh, T, d = q.shape
     D = packed_dim(d)
@@ -136,10 +146,24 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
     need = L.kata_prefill_workspace_bytes(B, Hh, T, d, chunk, dt)
     if workspace is None:
         workspace = _workspace(need, q.device)
-    _check("kata_prefill", L.kata_prefill(
+    _check("kata_prefill_ex", L.kata_prefill_ex(
         _ptr(q), _ptr(k), _ptr(v), dt, B, Hh, T, d, chunk, eps, _ptr(H_in), _ptr(s_in),
-        _ptr(o), _ptr(H_out), _ptr(s_out), _ptr(workspace), workspace.numel(), _stream(stream)))
+        _ptr(o), _ptr(H_out), _ptr(s_out), _ptr(workspace), workspace.numel(), _stream(stream),
+        FORMS[form]))
     return o, H_out, s_out
+
+
+def prefill_auto_form(B, H, T, d, chunk, dtype, output_only: bool) -> str:
+    """The form kata_prefill takes for these sizes: "chunked" or "quadratic"."""
+    f = int(lib().kata_prefill_auto_form(B, H, T, d, chunk, _DTYPE[dtype], int(output_only)))
+    if f < 0:
+        raise KataError(f"kata_prefill_auto_form: invalid arguments ({B}, {H}, {T}, {d}, {chunk})")
+    return "quadratic" if f == FORMS["quadratic"] else "chunked"
+
+
+def quadratic_max_tokens(d: int) -> int:
+    """Largest T for which kata_prefill takes the quadratic form (0: never)."""
+    return int(lib().kata_quadratic_max_tokens(d))
 
 
 def prefill_uses_tensor_cores(B, H, T, d, chunk, dtype) -> bool:

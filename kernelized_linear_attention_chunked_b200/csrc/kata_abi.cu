@@ -142,12 +142,48 @@ size_t kata_prefill_workspace_bytes(int B, int H, int T, int d, int chunk, int d
     return prefill_ws_bytes(B, H, T, d, chunk, dtype);
 }
 
+int kata_quadratic_max_tokens(int d) {
+    // measured crossover of the output-only prefill on B200: below it the
+    // quadratic form's O(T^2 d) work beats the chunked form's state carry
+    return d == 32 ? 4096 : d == 64 ? 2048 : 0;
+}
+
+static bool quadratic_applies(int dtype, int B, int H, int T, int d, bool output_only) {
+    kata::PrefillArgs a{};
+    a.dtype = dtype;
+    a.B = B;
+    a.H = H;
+    a.T = T;
+    a.d = d;
+    a.o = reinterpret_cast<float *>(16);  // alignment of the real pointers is checked later
+    a.q = a.k = a.v = a.o;
+    return output_only && dtype == KATA_BF16 && kata::quad_tc_supported(a);
+}
+
+int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int output_only) {
+    if (check_prefill(dtype, B, H, T, d, chunk)) return -1;
+    return quadratic_applies(dtype, B, H, T, d, output_only != 0) &&
+                   T <= kata_quadratic_max_tokens(d)
+               ? KATA_FORM_QUADRATIC
+               : KATA_FORM_CHUNKED;
+}
+
 int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
                  int d, int chunk, float eps, const float *H_in, const float *s_in, float *o,
                  float *H_out, float *s_out, void *workspace, size_t ws_bytes, void *stream) {
+    return kata_prefill_ex(q, k, v, dtype, B, H, T, d, chunk, eps, H_in, s_in, o, H_out, s_out,
+                           workspace, ws_bytes, stream, KATA_FORM_AUTO);
+}
+
+int kata_prefill_ex(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
+                    int d, int chunk, float eps, const float *H_in, const float *s_in, float *o,
+                    float *H_out, float *s_out, void *workspace, size_t ws_bytes, void *stream,
+                    int form) {
     g_last_error[0] = 0;
     int st = check_prefill(dtype, B, H, T, d, chunk);
     if (st) return st;
+    if (form != KATA_FORM_AUTO && form != KATA_FORM_CHUNKED && form != KATA_FORM_QUADRATIC)
+        return fail(KATA_ERR_INVALID_ARG, "form=%d: 0 (auto), 1 (chunked) or 2 (quadratic)", form);
     KATA_REQUIRE_PTR(q);
     KATA_REQUIRE_PTR(k);
     KATA_REQUIRE_PTR(v);
@@ -159,6 +195,23 @@ int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, 
     if (!H_in != !s_in) return fail(KATA_ERR_INVALID_ARG, "H_in and s_in: both or neither");
     if (!H_out != !s_out) return fail(KATA_ERR_INVALID_ARG, "H_out and s_out: both or neither");
     if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const bool output_only = o && !H_in && !H_out;
+    if (form == KATA_FORM_AUTO)
+        form = quadratic_applies(dtype, B, H, T, d, output_only) && T <= kata_quadratic_max_tokens(d)
+                   ? KATA_FORM_QUADRATIC
+                   : KATA_FORM_CHUNKED;
+    if (form == KATA_FORM_QUADRATIC) {
+        if (!quadratic_applies(dtype, B, H, T, d, output_only))
+            return fail(KATA_ERR_UNSUPPORTED,
+                        "quadratic form: bf16, d = 32 or 64, T a multiple of 128, o only");
+        unsigned int *err = error_word();
+        if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
+        kata::PrefillArgs a{q, k, v, dtype, B, H, T, d, chunk, eps, nullptr, nullptr, o,
+                            nullptr, nullptr, nullptr, 0, err};
+        cudaError_t e = kata::quad_tc(a, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "kata_prefill (quadratic form) launch");
+        return KATA_OK;
+    }
     const size_t need = prefill_ws_bytes(B, H, T, d, chunk, dtype);
     if (ws_bytes < need || (need && !workspace))
         return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);

@@ -27,6 +27,11 @@ bool prefill_tc_supported(const PrefillArgs &a);
 size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
 cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream);
 
+// tcgen05 quadratic form (bf16, d = 32 or 64, T a multiple of 128): o only,
+// from a zero state; H_in, H_out, ws are ignored.
+bool quad_tc_supported(const PrefillArgs &a);
+cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream);
+
 cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
                         int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream);
 

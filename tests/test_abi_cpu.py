@@ -5,6 +5,7 @@ import re
 from pathlib import Path
 
 import pytest
+import torch
 
 import kernelized_linear_attention_chunked_b200 as kata
 from kernelized_linear_attention_chunked_b200 import _binding
@@ -20,7 +21,7 @@ def header_functions():
 
 def test_header_symbols_exported_and_bound():
     names = header_functions()
-    assert len(names) == 20
+    assert len(names) == 23
     L = kata.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -86,6 +87,49 @@ def _prefill(**kw):
 ])
 def test_prefill_validation(kw, status):
     assert _prefill(**kw) == status
+    assert kata.lib().kata_last_error()
+
+
+def _prefill_ex(form, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, B=1, H=1, T=256, d=32, chunk=64, eps=1e-6,
+             H_in=None, s_in=None, o=FAKE, H_out=None, s_out=None, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return kata.lib().kata_prefill_ex(*a.values(), None, form)
+
+
+def test_prefill_form_selection():
+    L = kata.lib()
+    assert L.kata_quadratic_max_tokens(32) >= 2048
+    assert L.kata_quadratic_max_tokens(16) == 0
+    for d in (32, 64):
+        tmax = L.kata_quadratic_max_tokens(d)
+        assert tmax % 128 == 0
+        # output-only bf16 calls up to the crossover take the quadratic form
+        assert L.kata_prefill_auto_form(4, 8, tmax, d, 64, 1, 1) == 2
+        assert L.kata_prefill_auto_form(4, 8, tmax + 128, d, 64, 1, 1) == 1
+        # a call that reads or writes the state, fp32 inputs, or T % 128 != 0: chunked
+        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 1, 0) == 1
+        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 0, 1) == 1
+        assert L.kata_prefill_auto_form(4, 8, 192, d, 64, 1, 1) == 1
+    assert L.kata_prefill_auto_form(1, 1, 256, 16, 64, 1, 1) == 1
+    assert L.kata_prefill_auto_form(1, 1, 250, 32, 64, 1, 1) == -1
+    assert kata.prefill_auto_form(4, 8, 2048, 32, 64, torch.bfloat16, True) == "quadratic"
+    assert kata.prefill_auto_form(2, 16, 16384, 64, 128, torch.bfloat16, True) == "chunked"
+
+
+@pytest.mark.parametrize("form,kw,status", [
+    (7, {}, 1),                                    # no such form
+    (-1, {}, 1),
+    (2, dict(dtype=0), 2),                         # quadratic: bf16 only
+    (2, dict(d=16), 2),                            # quadratic: d = 32 or 64
+    (2, dict(T=192), 2),                           # quadratic: T a multiple of 128
+    (2, dict(o=None, H_out=FAKE, s_out=FAKE), 2),  # quadratic: output only
+    (2, dict(H_in=FAKE, s_in=FAKE), 2),
+    (2, dict(q=MISALIGNED), 1),
+    (1, dict(ws=None, ws_bytes=0), 5),             # the chunked form needs its workspace
+])
+def test_prefill_ex_validation(form, kw, status):
+    assert _prefill_ex(form, **kw) == status
     assert kata.lib().kata_last_error()
 
 
