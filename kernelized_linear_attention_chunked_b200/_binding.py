@@ -85,12 +85,12 @@ def _check(name: str, status: int) -> None:
 
 
 def _ptr(t):
-    return None if t is None else C.c_void_p(t.data_ptr())
+    return None if t is None else t.data_ptr()
 
 
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
-    return C.c_void_p(s.cuda_stream)
+    return s.cuda_stream
 
 
 def _dt(t: torch.Tensor) -> int:
@@ -135,7 +135,7 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
     ``form``: "chunked", "quadratic" (output only) or "auto" (kata_prefill's choice)."""
     _dev(q, k, v, H_in, s_in)
     B, Hh, T, d = q.shape
-    D = packed_dim(d)
+    D = d * (d + 1) // 2
     dt = _dt(q)
     if output and o is None:
         o = torch.empty(B, Hh, T, d, dtype=torch.float32, device=q.device)
@@ -143,13 +143,12 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
         H_out = torch.empty(B, Hh, D, d, dtype=torch.float32, device=q.device)
         s_out = torch.empty(B, Hh, D, dtype=torch.float32, device=q.device)
     L = lib()
-    need = L.kata_prefill_workspace_bytes(B, Hh, T, d, chunk, dt)
     if workspace is None:
-        workspace = _workspace(need, q.device)
+        workspace = _workspace(L.kata_prefill_workspace_bytes(B, Hh, T, d, chunk, dt), q.device)
     _check("kata_prefill_ex", L.kata_prefill_ex(
-        _ptr(q), _ptr(k), _ptr(v), dt, B, Hh, T, d, chunk, eps, _ptr(H_in), _ptr(s_in),
-        _ptr(o), _ptr(H_out), _ptr(s_out), _ptr(workspace), workspace.numel(), _stream(stream),
-        FORMS[form]))
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, B, Hh, T, d, chunk, eps, _ptr(H_in),
+        _ptr(s_in), _ptr(o), _ptr(H_out), _ptr(s_out), workspace.data_ptr(), workspace.numel(),
+        _stream(stream), FORMS[form]))
     return o, H_out, s_out
 
 

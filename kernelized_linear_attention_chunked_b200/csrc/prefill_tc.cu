@@ -807,11 +807,9 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
         // accumulators are narrow enough to keep two Phi(K)^T slots as well
         constexpr int NA = DH == 64 ? 1 : 2;
         using L = StateCfg<DH, 2, NA>;
-        auto kern = state_kernel<DH, 2, NA>;
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+        cudaError_t e = set_smem_once<state_kernel<DH, 2, NA>>(L::BYTES);
         if (e != cudaSuccess) return e;
-        kern<<<dim3(S::NT, nheads), L::THREADS, L::BYTES, stream>>>(mk, mv, sp);
+        state_kernel<DH, 2, NA><<<dim3(S::NT, nheads), L::THREADS, L::BYTES, stream>>>(mk, mv, sp);
         e = after_launch();
         if (e != cudaSuccess) return e;
     }
@@ -821,7 +819,7 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     constexpr int NIR = DH == 64 ? 1 : 2;
     using R = ReadCfg<DH, NIR>;
     auto kern = readout_kernel<DH, NIR>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, R::BYTES);
+    cudaError_t e = set_smem_once<readout_kernel<DH, NIR>>(R::BYTES);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: overlap this grid's setup and intra-chunk
     // work with the end of the state kernel

@@ -53,6 +53,20 @@ enum QuadBar {
     kQbCount = 18
 };
 
+// Square two fp32 scores (one packed f32x2 multiply, round to nearest) and
+// round the squares to a bf16 pair (first score in the low half).
+__device__ __forceinline__ uint32_t sq_pack(uint32_t x0, uint32_t x1) {
+    uint32_t d;
+    asm("{\n\t.reg .b64 a;\n\t.reg .f32 l, h;\n\t"
+        "mov.b64 a, {%1, %2};\n\t"
+        "mul.rn.f32x2 a, a, a;\n\t"
+        "mov.b64 {l, h}, a;\n\t"
+        "cvt.rn.bf16x2.f32 %0, h, l;\n\t}"
+        : "=r"(d)
+        : "r"(x0), "r"(x1));
+    return d;
+}
+
 template <int DH>
 struct QuadCfg {
     using S = Shape<DH>;
@@ -214,7 +228,7 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    pk[e] = pack_bf16x2(sv[2 * e] * sv[2 * e], sv[2 * e + 1] * sv[2 * e + 1]);
+                    pk[e] = sq_pack(__float_as_uint(sv[2 * e]), __float_as_uint(sv[2 * e + 1]));
             }
             if (j >= NP) warp_wait(&bar[kQbPFree + ps], (j / NP - 1) & 1, err, 0x621);
             tc_fence_after();
@@ -265,10 +279,9 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     if (!make_qkv_maps(&mq, &mk, &mv, a.q, a.k, a.v, DH, (long)nheads * a.T))
         return cudaErrorInvalidValue;
     QuadParams qp{nch, a.eps, a.o, a.err};
-    auto kern = quad_kernel<DH>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    cudaError_t e = set_smem_once<quad_kernel<DH>>(L::BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(nheads, nch), L::THREADS, L::BYTES, stream>>>(mq, mk, mv, qp);
+    quad_kernel<DH><<<dim3(nheads, nch), L::THREADS, L::BYTES, stream>>>(mq, mk, mv, qp);
     return after_launch();
 }
 

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "sm100.cuh"
@@ -85,6 +86,21 @@ inline PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
     });
     return fn;
+}
+
+// Raise `Kern`'s dynamic shared-memory limit to `bytes` once per device (the
+// attribute is per device; setting it on every launch costs host time).
+template <auto Kern>
+inline cudaError_t set_smem_once(int bytes) {
+    static std::atomic<unsigned long long> done{0};  // one bit per device ordinal < 64
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
 }
 
 // [rows, d] bf16 rows in boxes of 128 rows x box_x columns. Q and K use
