@@ -225,17 +225,18 @@ def time_events(fn, iters: int, stream) -> float:
 
 
 def per_launch_ms(fn, iters: int, stream) -> float:
-    """Mean duration of single calls, each bracketed by its own events."""
-    ts = []
+    """Mean device time of one call: CUDA events on `stream` around `iters`
+    back-to-back calls, divided by `iters`. (A call bracketed alone would also
+    count the host's launch preparation, during which the GPU idles.)"""
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
     for i in range(iters):
-        s = torch.cuda.Event(enable_timing=True)
-        e = torch.cuda.Event(enable_timing=True)
-        s.record(stream)
         fn(i)
-        e.record(stream)
-        e.synchronize()
-        ts.append(s.elapsed_time(e))
-    return float(np.mean(ts))
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / iters
 
 
 def barrier(dist_on):
@@ -320,7 +321,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
         else "simt"
     flops = quadratic_flops(w) if form == "quadratic" else prefill_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
-    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    lat = per_launch_ms(step, max(args.steps, 10), stream)
     chunked = None
     if form == "quadratic":
         # one launch per call: the quadratic-form kernel
@@ -417,7 +418,7 @@ def chunked_kernels(kata, w, sets, R, ws, args, stream, dev, lat_call):
 
     for i in range(3):
         state_step(i)
-    lat_state = per_launch_ms(state_step, max(args.steps, 5), stream)
+    lat_state = per_launch_ms(state_step, max(args.steps, 10), stream)
     lat_read = max(lat_call - lat_state, 1e-6)
     f_update = prefill_update_flops(w)
     f_read = flops - f_update
@@ -441,7 +442,7 @@ def bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks):
     for i in range(args.warmup):
         step(i)
     ms = time_events(step, args.steps, stream) / args.steps
-    lat = per_launch_ms(step, max(args.steps, 5), stream)
+    lat = per_launch_ms(step, max(args.steps, 10), stream)
     kata.sync_status()
     flops = prefill_flops(w)
     return {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),

@@ -145,7 +145,7 @@ size_t kata_prefill_workspace_bytes(int B, int H, int T, int d, int chunk, int d
 int kata_quadratic_max_tokens(int d) {
     // measured crossover of the output-only prefill on B200: below it the
     // quadratic form's O(T^2 d) work beats the chunked form's state carry
-    return d == 32 ? 4096 : d == 64 ? 2048 : 0;
+    return d == 32 ? 4096 : d == 64 ? 8192 : 0;
 }
 
 static bool quadratic_applies(int dtype, int B, int H, int T, int d, bool output_only) {
