@@ -149,15 +149,7 @@ int kata_quadratic_max_tokens(int d) {
 }
 
 static bool quadratic_applies(int dtype, int B, int H, int T, int d, bool output_only) {
-    kata::PrefillArgs a{};
-    a.dtype = dtype;
-    a.B = B;
-    a.H = H;
-    a.T = T;
-    a.d = d;
-    a.o = reinterpret_cast<float *>(16);  // alignment of the real pointers is checked later
-    a.q = a.k = a.v = a.o;
-    return output_only && dtype == KATA_BF16 && kata::quad_tc_supported(a);
+    return output_only && kata::quad_tc_shape_ok(dtype, B, H, T, d);
 }
 
 int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int output_only) {

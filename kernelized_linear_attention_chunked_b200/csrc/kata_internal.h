@@ -27,9 +27,10 @@ bool prefill_tc_supported(const PrefillArgs &a);
 size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int chunk);
 cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream);
 
-// tcgen05 quadratic form (bf16, d = 32 or 64, T a multiple of 128): o only,
-// from a zero state; H_in, H_out, ws are ignored.
-bool quad_tc_supported(const PrefillArgs &a);
+// tcgen05 quadratic form: o only, from a zero state; H_in, H_out, ws are
+// ignored. quad_tc_shape_ok tells the sizes it takes (bf16, d = 32 or 64, T a
+// multiple of 128); the caller checks that q, k, v, o are 16-byte aligned.
+bool quad_tc_shape_ok(int dtype, int B, int H, int T, int d);
 cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream);
 
 cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,

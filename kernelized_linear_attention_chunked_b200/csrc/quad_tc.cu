@@ -287,16 +287,14 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-bool quad_tc_supported(const PrefillArgs &a) {
-    return a.dtype == 1 && (a.d == 64 || a.d == 32) && a.T % kTile == 0 && a.T / kTile <= 65535 &&
-           (long)a.B * a.H * a.T < (1L << 31) && a.o != nullptr &&
-           (reinterpret_cast<uintptr_t>(a.q) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(a.k) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(a.v) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(a.o) & 15) == 0;
+bool quad_tc_shape_ok(int dtype, int B, int H, int T, int d) {
+    return dtype == 1 && (d == 64 || d == 32) && T > 0 && T % kTile == 0 &&
+           T / kTile <= 65535 && (long)B * H * T < (1L << 31) && (long)B * H <= 0x7FFFFFFFL;
 }
 
 cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream) {
+    if (!quad_tc_shape_ok(a.dtype, a.B, a.H, a.T, a.d) || a.o == nullptr)
+        return cudaErrorNotSupported;
     return a.d == 64 ? launch<64>(a, stream) : launch<32>(a, stream);
 }
 
