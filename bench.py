@@ -239,19 +239,41 @@ def per_launch_ms(fn, iters: int, stream) -> float:
     return s.elapsed_time(e) / iters
 
 
+def _sync_device():
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.synchronize()
+
+
 def barrier(dist_on):
-    torch.cuda.synchronize()
+    """Every rank's queued GPU work done, then a process-group barrier."""
+    _sync_device()
     if dist_on:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    _sync_device()
 
 
 def max_over_ranks(x: float, dist_on) -> float:
+    """The largest of the ranks' values (the slowest rank's time). The tensor
+    lives where the process group's backend reduces: the GPU for NCCL, the host
+    for gloo."""
     if not dist_on:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    nccl = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([x], device="cuda" if nccl else "cpu", dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes the same
+    per-GPU work, and the slowest rank's time (ms, max over ranks) bounds it."""
+    return world * units_per_step * steps / (ms / 1e3)
+
+
+def dist_env():
+    """(rank, world, local rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
 
 
 def run_kata(args, rank: int, world: int, dist_on: bool):
@@ -313,7 +335,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     kata.sync_status()
     ms = max_over_ranks(ms, dist_on)
     tokens_per_step = w.B * w.T
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = aggregate_rate(world, tokens_per_step, args.steps, ms)
     ms_step = ms / args.steps
     # the form kata_prefill takes for this output-only call, and its flops
     form = kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16, True)
@@ -370,7 +392,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
         e2e_step(i)
     barrier(dist_on)
     ms_e2e = max_over_ranks(time_events(e2e_step, args.steps, stream), dist_on)
-    e2e = {"value": world * tokens_per_step * args.steps / (ms_e2e / 1e3), "unit": "tokens/s",
+    e2e = {"value": aggregate_rate(world, tokens_per_step, args.steps, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
            "d2h_bytes_per_step": oh.numel() * 4}
     del sets, outs, qh, kh, vh, oh, wsh
@@ -481,7 +503,7 @@ def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
     kata.sync_status()
     ms_step = ms / nsteps
     gbs = decode_bytes(w) / (ms_step / 1e3) / 1e9
-    return {"workload": w.name, "tokens_per_s": world * w.B * nsteps / (ms / 1e3),
+    return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B, nsteps, ms),
             "us_per_step": 1e3 * ms_step, "steps": nsteps, "gbs": gbs,
             "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_step": decode_bytes(w),
             "gpu_launches": launches, "l2": "state 554 MB > 126 MB L2"}
@@ -547,7 +569,7 @@ def bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world):
     ms = max_over_ranks(time_events(step, n, stream), dist_on) / n
     kata.sync_status()
     fl = prefill_flops(w)
-    return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
+    return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B * w.T, 1, ms), "ms": ms,
             "tflops": fl / (ms / 1e3) / 1e12, "frac_bf16_peak": fl / (ms / 1e3) / 1e12 /
             peaks["bf16_tflops"], "l2": "inputs 335 MB > 126 MB L2"}
 
@@ -594,13 +616,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    rank, world, local = dist_env()
     dist_on = world > 1
     if args.impl == "reference":
         run_reference(args, rank)
         return
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     if dist_on:
         import datetime
