@@ -338,7 +338,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     value = aggregate_rate(world, tokens_per_step, args.steps, ms)
     ms_step = ms / args.steps
     # the form kata_prefill takes for this output-only call, and its flops
-    form = kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16, True)
+    form = kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16)
     path = "tc" if kata.prefill_uses_tensor_cores(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16) \
         else "simt"
     flops = quadratic_flops(w) if form == "quadratic" else prefill_flops(w)

@@ -127,18 +127,23 @@ enum { KATA_FORM_AUTO = 0, KATA_FORM_CHUNKED = 1, KATA_FORM_QUADRATIC = 2 };
 /*
  * kata_prefill with the form chosen by the caller.
  *   KATA_FORM_CHUNKED    the chunked state form described at kata_prefill.
- *   KATA_FORM_QUADRATIC  the quadratic form [KATA s2.2: the rank-one PSD
+ *   KATA_FORM_QUADRATIC  o by the quadratic form [KATA s2.2: the rank-one PSD
  *                        feature makes the kernel (q.k)^2]:
  *                          o_i = sum_{j<=i} (q_i.k_j)^2 v_j / (sum_{j<=i} (q_i.k_j)^2 + eps),
  *                        O(T^2 d) work on the tcgen05 tensor cores with no
  *                        state (bf16 (q.k)^2 operands, fp32 accumulation). It
  *                        takes bf16 inputs, d = 32 or 64, T a multiple of 128,
- *                        o non-NULL and H_in, s_in, H_out, s_out NULL; other
- *                        calls return KATA_ERR_UNSUPPORTED. workspace is not
- *                        used (may be NULL, ws_bytes 0).
- *   KATA_FORM_AUTO       what kata_prefill does: the quadratic form when it
- *                        applies and T <= kata_quadratic_max_tokens(d), the
- *                        chunked form otherwise.
+ *                        o non-NULL and H_in, s_in NULL; other calls return
+ *                        KATA_ERR_UNSUPPORTED. With H_out, s_out the final
+ *                        state is computed by the chunked form's state pass
+ *                        at the same time, on a second stream the library
+ *                        forks from `stream` and joins back to it with events
+ *                        (one per device, shared by the calling threads).
+ *                        workspace is not used (may be NULL, ws_bytes 0).
+ *   KATA_FORM_AUTO       what kata_prefill does: the quadratic form for a call
+ *                        without H_in and H_out when it applies and
+ *                        T <= kata_quadratic_max_tokens(d), the chunked form
+ *                        otherwise.
  * Both forms give the same result up to rounding.
  */
 KATA_API int kata_prefill_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
@@ -150,9 +155,10 @@ KATA_API int kata_prefill_ex(const void *q, const void *k, const void *v, int dt
 KATA_API int kata_quadratic_max_tokens(int d);
 
 /* The form KATA_FORM_AUTO takes for these sizes: KATA_FORM_CHUNKED or
- * KATA_FORM_QUADRATIC; output_only = o given, no initial or final state.
- * -1 = invalid or unsupported arguments. */
-KATA_API int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int output_only);
+ * KATA_FORM_QUADRATIC; with_state = H_in or H_out given (such calls take the
+ * chunked form). -1 = invalid or unsupported arguments. */
+KATA_API int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype,
+                                    int with_state);
 
 /* Device workspace for kata_prefill_host: staging for q, k, v and o plus
  * kata_prefill_workspace_bytes(). */

@@ -132,7 +132,9 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
             form: str = "auto"):
     """Causal prefill. q, k, v [B, H, T, d]. Returns (o, H, s); o is None when
     ``output`` is False (state only), H and s are None when ``state`` is False.
-    ``form``: "chunked", "quadratic" (output only) or "auto" (kata_prefill's choice)."""
+    ``form``: "chunked", "quadratic" (o from a zero initial state; the final
+    state, if asked for, by the state pass at the same time) or "auto"
+    (kata_prefill's choice)."""
     _dev(q, k, v, H_in, s_in)
     B, Hh, T, d = q.shape
     D = d * (d + 1) // 2
@@ -152,9 +154,10 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
     return o, H_out, s_out
 
 
-def prefill_auto_form(B, H, T, d, chunk, dtype, output_only: bool) -> str:
-    """The form kata_prefill takes for these sizes: "chunked" or "quadratic"."""
-    f = int(lib().kata_prefill_auto_form(B, H, T, d, chunk, _DTYPE[dtype], int(output_only)))
+def prefill_auto_form(B, H, T, d, chunk, dtype, with_state: bool = False) -> str:
+    """The form kata_prefill takes for these sizes: "chunked" or "quadratic"
+    (the latter only for calls without an initial or final state)."""
+    f = int(lib().kata_prefill_auto_form(B, H, T, d, chunk, _DTYPE[dtype], int(with_state)))
     if f < 0:
         raise KataError(f"kata_prefill_auto_form: invalid arguments ({B}, {H}, {T}, {d}, {chunk})")
     return "quadratic" if f == FORMS["quadratic"] else "chunked"

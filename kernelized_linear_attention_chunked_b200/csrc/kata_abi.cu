@@ -1,6 +1,7 @@
 // C ABI of libkata.so: argument validation, dispatch, status reporting.
 // The declarations and the contract of every entry point are in include/kata.h.
 #include <atomic>
+#include <mutex>
 #include <stdarg.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -43,6 +44,36 @@ unsigned int *error_word() {
 }
 
 std::atomic<unsigned long long> g_launches{0};
+
+// A second stream per device for work that runs beside the caller's stream
+// within one call, forked from and joined back to it with events.
+struct SideStream {
+    std::mutex mu;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream *side_stream() {
+    static SideStream sides[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    SideStream &sd = sides[dev];
+    std::lock_guard<std::mutex> lock(sd.mu);
+    if (!sd.stream) {
+        cudaStream_t st = nullptr;
+        cudaEvent_t f = nullptr, j = nullptr;
+        if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+            cudaStreamDestroy(st);
+            return nullptr;
+        }
+        sd.stream = st;
+        sd.fork = f;
+        sd.join = j;
+    }
+    return &sd;
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -148,16 +179,61 @@ int kata_quadratic_max_tokens(int d) {
     return d == 32 ? 4096 : d == 64 ? 8192 : 0;
 }
 
-static bool quadratic_applies(int dtype, int B, int H, int T, int d, bool output_only) {
-    return output_only && kata::quad_tc_shape_ok(dtype, B, H, T, d);
+// The quadratic form computes o from a zero initial state.
+static bool quadratic_applies(int dtype, int B, int H, int T, int d, bool from_initial_state) {
+    return !from_initial_state && kata::quad_tc_shape_ok(dtype, B, H, T, d);
 }
 
-int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int output_only) {
+// KATA_FORM_AUTO: the quadratic form for output-only calls up to the
+// crossover. With a final state the chunked form stays: running the state pass
+// beside the quadratic kernel measured no faster at d = 32 (57 vs 56 us at
+// B4 H8 T2048) and only wins at d = 64 for short T.
+static bool auto_quadratic(int dtype, int B, int H, int T, int d, bool with_state) {
+    return !with_state && quadratic_applies(dtype, B, H, T, d, false) &&
+           T <= kata_quadratic_max_tokens(d);
+}
+
+int kata_prefill_auto_form(int B, int H, int T, int d, int chunk, int dtype, int with_state) {
     if (check_prefill(dtype, B, H, T, d, chunk)) return -1;
-    return quadratic_applies(dtype, B, H, T, d, output_only != 0) &&
-                   T <= kata_quadratic_max_tokens(d)
-               ? KATA_FORM_QUADRATIC
-               : KATA_FORM_CHUNKED;
+    return auto_quadratic(dtype, B, H, T, d, with_state != 0) ? KATA_FORM_QUADRATIC
+                                                              : KATA_FORM_CHUNKED;
+}
+
+// o by the quadratic form; with H_out, the final state by the chunked form's
+// state kernel (no snapshots) on the side stream at the same time.
+static int prefill_quadratic(const void *q, const void *k, const void *v, int dtype, int B,
+                             int H, int T, int d, int chunk, float eps, float *o, float *H_out,
+                             float *s_out, cudaStream_t s) {
+    unsigned int *err = error_word();
+    if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
+    kata::PrefillArgs a{q, k, v, dtype, B, H, T, d, chunk, eps, nullptr, nullptr, o,
+                        nullptr, nullptr, nullptr, 0, err};
+    if (!H_out) {
+        cudaError_t e = kata::quad_tc(a, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kata_prefill (quadratic form) launch");
+        return KATA_OK;
+    }
+    kata::PrefillArgs st{q, k, v, dtype, B, H, T, d, chunk, eps, nullptr, nullptr, nullptr,
+                         H_out, s_out, nullptr, 0, err};
+    if (!kata::prefill_tc_supported(st))
+        return fail(KATA_ERR_UNSUPPORTED, "final state beside the quadratic form: not supported");
+    SideStream *sd = side_stream();
+    if (!sd) return fail(KATA_ERR_CUDA, "side stream unavailable");
+    cudaError_t e;
+    {
+        std::lock_guard<std::mutex> lock(sd->mu);
+        if ((e = cudaEventRecord(sd->fork, s)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(sd->stream, sd->fork, 0)) != cudaSuccess)
+            return cuda_fail(e, "fork to the side stream");
+        e = kata::prefill_tc(st, sd->stream);
+        cudaError_t ej = cudaEventRecord(sd->join, sd->stream);
+        if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, sd->join, 0);
+        if (e != cudaSuccess) return cuda_fail(e, "kata_prefill (state kernel) launch");
+        if (ej != cudaSuccess) return cuda_fail(ej, "join from the side stream");
+    }
+    e = kata::quad_tc(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_prefill (quadratic form) launch");
+    return KATA_OK;
 }
 
 int kata_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
@@ -187,22 +263,16 @@ int kata_prefill_ex(const void *q, const void *k, const void *v, int dtype, int 
     if (!H_in != !s_in) return fail(KATA_ERR_INVALID_ARG, "H_in and s_in: both or neither");
     if (!H_out != !s_out) return fail(KATA_ERR_INVALID_ARG, "H_out and s_out: both or neither");
     if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
-    const bool output_only = o && !H_in && !H_out;
+    const bool init = H_in != nullptr;
     if (form == KATA_FORM_AUTO)
-        form = quadratic_applies(dtype, B, H, T, d, output_only) && T <= kata_quadratic_max_tokens(d)
-                   ? KATA_FORM_QUADRATIC
-                   : KATA_FORM_CHUNKED;
+        form = o && auto_quadratic(dtype, B, H, T, d, init || H_out) ? KATA_FORM_QUADRATIC
+                                                                      : KATA_FORM_CHUNKED;
     if (form == KATA_FORM_QUADRATIC) {
-        if (!quadratic_applies(dtype, B, H, T, d, output_only))
-            return fail(KATA_ERR_UNSUPPORTED,
-                        "quadratic form: bf16, d = 32 or 64, T a multiple of 128, o only");
-        unsigned int *err = error_word();
-        if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
-        kata::PrefillArgs a{q, k, v, dtype, B, H, T, d, chunk, eps, nullptr, nullptr, o,
-                            nullptr, nullptr, nullptr, 0, err};
-        cudaError_t e = kata::quad_tc(a, static_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return cuda_fail(e, "kata_prefill (quadratic form) launch");
-        return KATA_OK;
+        if (!o || !quadratic_applies(dtype, B, H, T, d, init))
+            return fail(KATA_ERR_UNSUPPORTED, "quadratic form: bf16, d = 32 or 64, T a multiple "
+                                              "of 128, o given, no initial state");
+        return prefill_quadratic(q, k, v, dtype, B, H, T, d, chunk, eps, o, H_out, s_out,
+                                 static_cast<cudaStream_t>(stream));
     }
     const size_t need = prefill_ws_bytes(B, H, T, d, chunk, dtype);
     if (ws_bytes < need || (need && !workspace))

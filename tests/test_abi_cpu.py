@@ -105,16 +105,17 @@ def test_prefill_form_selection():
         tmax = L.kata_quadratic_max_tokens(d)
         assert tmax % 128 == 0
         # output-only bf16 calls up to the crossover take the quadratic form
-        assert L.kata_prefill_auto_form(4, 8, tmax, d, 64, 1, 1) == 2
-        assert L.kata_prefill_auto_form(4, 8, tmax + 128, d, 64, 1, 1) == 1
-        # a call that reads or writes the state, fp32 inputs, or T % 128 != 0: chunked
-        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 1, 0) == 1
-        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 0, 1) == 1
-        assert L.kata_prefill_auto_form(4, 8, 192, d, 64, 1, 1) == 1
-    assert L.kata_prefill_auto_form(1, 1, 256, 16, 64, 1, 1) == 1
-    assert L.kata_prefill_auto_form(1, 1, 250, 32, 64, 1, 1) == -1
-    assert kata.prefill_auto_form(4, 8, 2048, 32, 64, torch.bfloat16, True) == "quadratic"
-    assert kata.prefill_auto_form(2, 16, 16384, 64, 128, torch.bfloat16, True) == "chunked"
+        assert L.kata_prefill_auto_form(4, 8, tmax, d, 64, 1, 0) == 2
+        assert L.kata_prefill_auto_form(4, 8, tmax + 128, d, 64, 1, 0) == 1
+        # with an initial or final state, fp32 inputs, or T % 128 != 0: chunked
+        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 1, 1) == 1
+        assert L.kata_prefill_auto_form(4, 8, 1024, d, 64, 0, 0) == 1
+        assert L.kata_prefill_auto_form(4, 8, 192, d, 64, 1, 0) == 1
+    assert L.kata_prefill_auto_form(1, 1, 256, 16, 64, 1, 0) == 1
+    assert L.kata_prefill_auto_form(1, 1, 250, 32, 64, 1, 0) == -1
+    assert kata.prefill_auto_form(4, 8, 2048, 32, 64, torch.bfloat16) == "quadratic"
+    assert kata.prefill_auto_form(4, 8, 2048, 32, 64, torch.bfloat16, True) == "chunked"
+    assert kata.prefill_auto_form(2, 16, 16384, 64, 128, torch.bfloat16) == "chunked"
 
 
 @pytest.mark.parametrize("form,kw,status", [
@@ -123,8 +124,8 @@ def test_prefill_form_selection():
     (2, dict(dtype=0), 2),                         # quadratic: bf16 only
     (2, dict(d=16), 2),                            # quadratic: d = 32 or 64
     (2, dict(T=192), 2),                           # quadratic: T a multiple of 128
-    (2, dict(o=None, H_out=FAKE, s_out=FAKE), 2),  # quadratic: output only
-    (2, dict(H_in=FAKE, s_in=FAKE), 2),
+    (2, dict(o=None, H_out=FAKE, s_out=FAKE), 2),  # quadratic: o is required
+    (2, dict(H_in=FAKE, s_in=FAKE), 2),             # quadratic: zero initial state only
     (2, dict(q=MISALIGNED), 1),
     (1, dict(ws=None, ws_bytes=0), 5),             # the chunked form needs its workspace
 ])

@@ -16,7 +16,9 @@ BF16 = torch.bfloat16
 
 
 def run(q, k, v, **kw):
-    out = kata.prefill(*cuda(q, k, v), chunk=64, **kw)
+    # the chunked form (kata_prefill would compute o by the quadratic form at
+    # these sizes when no initial state is given)
+    out = kata.prefill(*cuda(q, k, v), chunk=64, form="chunked", **kw)
     kata.sync_status()
     return out
 

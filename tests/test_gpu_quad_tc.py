@@ -1,7 +1,7 @@
 """The tcgen05 quadratic form (kata_prefill_ex, KATA_FORM_QUADRATIC, and the
-output-only calls kata_prefill routes to it) against the fp64 oracle's plain
-definition o_i = sum_{j<=i} (q_i.k_j)^2 v_j / (sum_{j<=i} (q_i.k_j)^2 + eps)
-(GPU)."""
+output-only calls kata_prefill routes to it) against the fp64 oracle's
+plain definition o_i = sum_{j<=i} (q_i.k_j)^2 v_j / (sum_{j<=i} (q_i.k_j)^2 + eps),
+and the final state that the state pass computes beside it (GPU)."""
 import numpy as np
 import pytest
 import torch
@@ -78,25 +78,64 @@ def test_first_token_and_eps():
 
 def test_auto_form_routes_output_only_calls():
     B, H, T, d = 1, 2, 256, 32
-    assert kata.prefill_auto_form(B, H, T, d, 64, BF16, True) == "quadratic"
+    assert kata.prefill_auto_form(B, H, T, d, 64, BF16) == "quadratic"
     q, k, v = prefill_inputs(B, H, T, d, dtype="bf16", seed=31)
     n0 = kata.launch_count()
     o, _, _ = kata.prefill(*cuda(q, k, v), chunk=64, state=False)
     kata.sync_status()
     assert kata.launch_count() - n0 == 1  # one kernel: the quadratic form
     assert rel_l2(o, oracle.quadratic(q, k, v, 1e-6)) < tol("bf16")
-    # with the state requested the chunked form runs (two kernels)
+    # with the final state requested kata_prefill takes the chunked form (the
+    # state kernel and the readout kernel)
+    assert kata.prefill_auto_form(B, H, T, d, 64, BF16, with_state=True) == "chunked"
     n0 = kata.launch_count()
     kata.prefill(*cuda(q, k, v), chunk=64)
     kata.sync_status()
     assert kata.launch_count() - n0 == 2
 
 
-def test_quadratic_form_rejects_state_arguments():
+# output and final state together: o by the quadratic form on the caller's
+# stream, (H, s) by the state pass on the side stream, joined back
+@pytest.mark.parametrize("d,T", [(32, 128), (32, 1024), (64, 640), (64, 2048)])
+def test_output_and_final_state(d, T):
+    q, k, v = prefill_inputs(2, 3, T, d, dtype="bf16", seed=50 + d + T)
+    o, H, s = kata.prefill(*cuda(q, k, v), chunk=64, form="quadratic")
+    kata.sync_status()
+    ro, rH, rs = oracle.recurrent(q, k, v, 1e-6)
+    assert rel_l2(o, ro) < tol("bf16")
+    assert rel_l2(H, rH) < tol("bf16")
+    assert rel_l2(s, rs) < tol("bf16")
+    # the same state as the chunked form's state pass computes (bit for bit)
+    _, H2, s2 = kata.prefill(*cuda(q, k, v), chunk=64, form="chunked")
+    kata.sync_status()
+    assert torch.equal(H, H2) and torch.equal(s, s2)
+
+
+def test_final_state_is_joined_back_to_the_callers_stream():
+    # a kernel queued on the caller's stream right after the call must see the
+    # final state: read it on that stream before any host synchronisation
+    q, k, v = cuda(*prefill_inputs(1, 4, 1024, 64, dtype="bf16", seed=8))
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        o, H, s = kata.prefill(q, k, v, chunk=64, form="quadratic", stream=stream)
+        snapshot = H.clone()  # enqueued on `stream` after the call
+    stream.synchronize()
+    kata.sync_status()
+    assert torch.equal(snapshot, H)
+    _, rH, _ = oracle.recurrent(q.cpu(), k.cpu(), v.cpu(), 1e-6, readout=False)
+    assert rel_l2(snapshot, rH) < tol("bf16")
+
+
+def test_quadratic_form_rejects_what_it_cannot_take():
     q, k, v = cuda(*prefill_inputs(1, 1, 128, 32, dtype="bf16", seed=1))
-    with pytest.raises(kata.KataError):
-        kata.prefill(q, k, v, chunk=64, state=True, form="quadratic")
-    with pytest.raises(kata.KataError):
+    D = 32 * 33 // 2
+    H0 = torch.zeros(1, 1, D, 32, device="cuda")
+    s0 = torch.zeros(1, 1, D, device="cuda")
+    with pytest.raises(kata.KataError):  # an initial state
+        kata.prefill(q, k, v, chunk=64, H_in=H0, s_in=s0, form="quadratic")
+    with pytest.raises(kata.KataError):  # no output
+        kata.prefill(q, k, v, chunk=64, output=False, form="quadratic")
+    with pytest.raises(kata.KataError):  # fp32 inputs
         kata.prefill(q.float(), k.float(), v.float(), chunk=64, state=False, form="quadratic")
 
 
@@ -104,7 +143,7 @@ def test_full_size_headline_config():
     # B4 H8 T2048 d32 output-only, as the headline step runs it; sampled rows
     # of every head against the oracle, computed row by row
     w = WORKLOADS["prefill_b4_h8_t2048_d32"]
-    assert kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, BF16, True) == "quadratic"
+    assert kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, BF16) == "quadratic"
     q, k, v = prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed, recipe=w.recipe)
     o, _, _ = kata.prefill(*cuda(q, k, v), chunk=w.chunk, eps=w.eps, state=False)
     kata.sync_status()
