@@ -88,6 +88,10 @@ struct StateParams {
     int nch;        // chunks per head
     int cpi;        // chunks per snapshot interval
     int nint;       // snapshot intervals per head
+    int seg_len;    // chunks per sequence segment (grid z): segment z starts at
+                    // chunk z * seg_len; with several segments there are no
+                    // snapshots and segment z writes its own partial state at
+                    // H_out + z * heads * D * d, s_out + z * heads * D
     const float *H_in, *s_in;
     float *H_out, *s_out;
     uint8_t *snap;  // [heads][nint][NS][NSNAP][128 B], or null: no snapshots
@@ -174,7 +178,15 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const long row0 = (long)head * p.nch * kTile;  // first token row of this head
+    // this CTA's chunks: [c0, c0 + nch) of its head
+    const int c0 = (int)blockIdx.z * p.seg_len;
+    const int nch = p.nch - c0 < p.seg_len ? p.nch - c0 : p.seg_len;
+    const long row0 = ((long)head * p.nch + c0) * kTile;  // first token row of this CTA
+    constexpr int D = DH * (DH + 1) / 2;
+    float *H_out = p.H_out ? p.H_out + (size_t)blockIdx.z * gridDim.y * D * DH : nullptr;
+    float *s_out = p.s_out ? p.s_out + (size_t)blockIdx.z * gridDim.y * D : nullptr;
+    // the initial state enters through the first segment only
+    const float *H_in = blockIdx.z == 0 ? p.H_in : nullptr;
     // the readout kernel may start its setup and intra-chunk work now; it waits
     // for this grid's completion before it reads a snapshot
     if (threadIdx.x == 0) launch_dependents();
@@ -188,9 +200,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             // workers, the MMAs): issue whichever slot frees first
             int nk = 0, nv = 0;
             uint32_t idle = 0;
-            while ((nk < p.nch || nv < p.nch) && idle < (1u << 24)) {
+            while ((nk < nch || nv < nch) && idle < (1u << 24)) {
                 bool moved = false;
-                if (nk < p.nch) {
+                if (nk < nch) {
                     const int ks = nk % L::KR, kn = nk / L::KR;
                     if (kn == 0 || mbar_test_wait(&bar[kSbKFree + ks], (kn - 1) & 1)) {
                         mbar_arrive_expect_tx(&bar[kSbKFull + ks], kTileBytes);
@@ -200,7 +212,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                         moved = true;
                     }
                 }
-                if (nv < p.nch) {
+                if (nv < nch) {
                     const int s = nv & 1, n = nv >> 1;
                     if (n == 0 || mbar_test_wait(&bar[kSbVFree + s], (n - 1) & 1)) {
                         mbar_arrive_expect_tx(&bar[kSbVFull + s], S::VBYTES);
@@ -215,11 +227,11 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                     if ((++idle & 1023u) == 0u && *((volatile unsigned int *)err) != 0u) break;
                 }
             }
-            if (nk < p.nch || nv < p.nch) atomicCAS(err, 0u, 0x401u);
+            if (nk < nch || nv < nch) atomicCAS(err, 0u, 0x401u);
             // no copy may still be in flight when the CTA exits
-            for (int c = p.nch - L::KR < 0 ? 0 : p.nch - L::KR; c < p.nch; ++c)
+            for (int c = nch - L::KR < 0 ? 0 : nch - L::KR; c < nch; ++c)
                 mbar_wait(&bar[kSbKFull + c % L::KR], (c / L::KR) & 1, err, 0x403);
-            for (int c = p.nch - 2 < 0 ? 0 : p.nch - 2; c < p.nch; ++c)
+            for (int c = nch - 2 < 0 ? 0 : nch - 2; c < nch; ++c)
                 mbar_wait(&bar[kSbVFull + (c & 1)], (c >> 1) & 1, err, 0x404);
         }
     } else if (warp >= 4) {
@@ -229,7 +241,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             const uint32_t idesc = idesc_bf16(128, S::NACC, 0, 1);
             const uint32_t ones = smem_u32(sm + L::ONES);
             const uint32_t acc = tmem + L::acc_col(ii);
-            for (int c = 0; c < p.nch; ++c) {
+            for (int c = 0; c < nch; ++c) {
                 const int s = c & 1, sa = c % NA;
                 mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412);
                 mbar_wait(&bar[kSbAFull + sa], (c / NA) & 1, err, 0x410);
@@ -274,12 +286,12 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
         // initial state: H_in in the internal scaling (no sqrt 2) in accumulator 0
         float init[DH + 1];
         {
-            const bool have = valid && p.H_in != nullptr;
+            const bool have = valid && H_in != nullptr;
             const int ci = valid ? canon_index(ra, rb, DH) : 0;
             const float w = (ra != rb) ? 0.70710678118654752f : 1.f;
             const size_t hb = ((size_t)head * (DH * (DH + 1) / 2) + ci);
 #pragma unroll
-            for (int n = 0; n < DH; ++n) init[n] = have ? p.H_in[hb * DH + n] * w : 0.f;
+            for (int n = 0; n < DH; ++n) init[n] = have ? H_in[hb * DH + n] * w : 0.f;
             init[DH] = have ? p.s_in[hb] * w : 0.f;
             uint32_t r[16];
 #pragma unroll
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                                         S::SLICE_BYTES,
                            stage, nvalid * S::SLICE_BYTES);
         };
-        if (p.H_in) write_snapshot(0, init);
+        if (H_in) write_snapshot(0, init);
         if (f == 0) bulk_wait_read();
         // the state: sum of the issuers' accumulators, columns 0..DH-1 and s
         auto read_acc = [&](float (&x)[DH + 1]) {
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
         };
 
         constexpr int NCB = DH / 8;  // 8-column blocks of a K row
-        for (int c = 0; c < p.nch; ++c) {
+        for (int c = 0; c < nch; ++c) {
             const int sa = c % NA, ks = c % L::KR;
             // transpose the K tile in 8 x 8 blocks (8 tokens x 8 columns per thread)
             warp_wait(&bar[kSbKFull + ks], (c / L::KR) & 1, err, 0x420);
@@ -416,21 +428,21 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             }
         }
         // final state, converted to the canonical layout
-        warp_wait(&bar[kSbDone + (p.nch - 1) % NA], ((p.nch - 1) / NA) & 1, err, 0x423);
+        warp_wait(&bar[kSbDone + (nch - 1) % NA], ((nch - 1) / NA) & 1, err, 0x423);
         tc_fence_after();
-        if (p.H_out) {
+        if (H_out) {
             float fin[DH + 1];
             read_acc(fin);
             if (valid && ra <= rb) {
                 const int ci = canon_index(ra, rb, DH);
                 const float w = (ra != rb) ? 1.41421356237309505f : 1.f;
                 const size_t hb = (size_t)head * (DH * (DH + 1) / 2) + ci;
-                float4 *dst = reinterpret_cast<float4 *>(p.H_out + hb * DH);
+                float4 *dst = reinterpret_cast<float4 *>(H_out + hb * DH);
 #pragma unroll
                 for (int n = 0; n < DH; n += 4)
                     dst[n / 4] = make_float4(fin[n] * w, fin[n + 1] * w, fin[n + 2] * w,
                                              fin[n + 3] * w);
-                p.s_out[hb] = fin[DH] * w;
+                s_out[hb] = fin[DH] * w;
             }
         }
         if (f == 0) bulk_wait_all();
@@ -789,6 +801,52 @@ size_t snapshot_bytes(long nheads, int nch) {
     return (size_t)nheads * nint * Shape<DH>::NS * Shape<DH>::SLICE_BYTES;
 }
 
+// Sequence segments of a final-state-only pass: as many (tile, head, segment)
+// CTAs as fit in one wave of two per SM (a second, partial wave costs more than
+// the split saves), at most 8 segments and one chunk per segment.
+int state_segments(int d, long nheads, int nch) {
+    const long ctas = (long)(d == 64 ? Shape<64>::NT : Shape<32>::NT) * nheads;
+    long seg = (2 * 148) / ctas;
+    if (seg > 8) seg = 8;
+    if (seg > nch) seg = nch;
+    return seg < 1 ? 1 : (int)seg;
+}
+
+// Partial states of the segments: H then s of each segment, 256-byte aligned.
+size_t partial_state_bytes(int d, long nheads, int nseg) {
+    if (nseg <= 1) return 0;
+    const size_t D = (size_t)d * (d + 1) / 2;
+    return align_up((size_t)nseg * nheads * D * d * 4, 256) +
+           align_up((size_t)nseg * nheads * D * 4, 256);
+}
+
+// out[i] = sum over the segments z = 0, 1, ... of part[z * n + i] (in that
+// order), four floats per thread.
+__global__ void __launch_bounds__(256) state_sum_kernel(const float4 *__restrict__ part, int nseg,
+                                                        long n4, float4 *__restrict__ out) {
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
+         i += (long)gridDim.x * blockDim.x) {
+        float4 acc = part[i];
+        for (int z = 1; z < nseg; ++z) {
+            const float4 x = part[(size_t)z * n4 + i];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        out[i] = acc;
+    }
+}
+
+cudaError_t launch_state_sum(const float *part, int nseg, size_t n, float *out,
+                             cudaStream_t stream) {
+    const long n4 = (long)(n / 4);
+    const int blocks = (int)((n4 + 255) / 256 < 4 * 148 ? (n4 + 255) / 256 : 4 * 148);
+    state_sum_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4 *>(part), nseg,
+                                                 n4, reinterpret_cast<float4 *>(out));
+    return after_launch();
+}
+
 template <int DH>
 cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     using S = Shape<DH>;
@@ -801,7 +859,29 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     if (!make_qkv_maps(&mq, &mk, &mv, a.q, a.k, a.v, DH, rows)) return cudaErrorInvalidValue;
 
-    StateParams sp{nch, cpi, nint, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
+    StateParams sp{nch, cpi, nint, nch, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
+    // a final-state-only pass: no interval ends inside the chunk loop, and the
+    // sequence split into segments when the tiles alone leave SMs idle (their
+    // partial states summed afterwards), if the workspace holds the partials
+    int nseg = 1;
+    float *pH = nullptr, *ps = nullptr;
+    if (!want_o) {
+        sp.cpi = nch;
+        sp.nint = 1;
+        const int want = state_segments(DH, nheads, nch);
+        if (want > 1 && a.H_out && a.ws &&
+            a.ws_bytes >= partial_state_bytes(DH, nheads, want)) {
+            nseg = want;
+            sp.seg_len = (nch + nseg - 1) / nseg;
+            nseg = (nch + sp.seg_len - 1) / sp.seg_len;  // no empty segment
+            const size_t D = (size_t)DH * (DH + 1) / 2;
+            pH = static_cast<float *>(a.ws);
+            ps = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) +
+                                           align_up((size_t)nseg * nheads * D * DH * 4, 256));
+            sp.H_out = pH;
+            sp.s_out = ps;
+        }
+    }
     {
         // two issuers halve the MMA issue chain of a chunk; with d = 32 the
         // accumulators are narrow enough to keep two Phi(K)^T slots as well
@@ -809,8 +889,16 @@ cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
         using L = StateCfg<DH, 2, NA>;
         cudaError_t e = set_smem_once<state_kernel<DH, 2, NA>>(L::BYTES);
         if (e != cudaSuccess) return e;
-        state_kernel<DH, 2, NA><<<dim3(S::NT, nheads), L::THREADS, L::BYTES, stream>>>(mk, mv, sp);
+        state_kernel<DH, 2, NA><<<dim3(S::NT, nheads, nseg), L::THREADS, L::BYTES, stream>>>(
+            mk, mv, sp);
         e = after_launch();
+        if (e != cudaSuccess) return e;
+    }
+    if (nseg > 1) {
+        const size_t D = (size_t)DH * (DH + 1) / 2;
+        cudaError_t e = launch_state_sum(pH, nseg, (size_t)nheads * D * DH, a.H_out, stream);
+        if (e != cudaSuccess) return e;
+        e = launch_state_sum(ps, nseg, (size_t)nheads * D, a.s_out, stream);
         if (e != cudaSuccess) return e;
     }
     if (!want_o) return cudaSuccess;
@@ -850,10 +938,12 @@ bool prefill_tc_supported(const PrefillArgs &a) {
 }
 
 size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int) {
-    if (T % kTile) return 0;
-    if (d == 32) return snapshot_bytes<32>((long)B * H, T / kTile);
-    if (d == 64) return snapshot_bytes<64>((long)B * H, T / kTile);
-    return 0;
+    if (T % kTile || (d != 32 && d != 64)) return 0;
+    const long nheads = (long)B * H;
+    const int nch = T / kTile;
+    const size_t snaps = d == 32 ? snapshot_bytes<32>(nheads, nch) : snapshot_bytes<64>(nheads, nch);
+    const size_t parts = partial_state_bytes(d, nheads, state_segments(d, nheads, nch));
+    return snaps > parts ? snaps : parts;
 }
 
 cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream) {

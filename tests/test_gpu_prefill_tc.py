@@ -46,9 +46,13 @@ def test_output_and_state(d, T):
     assert rel_l2(o, ro) < tol("bf16")
     assert rel_l2(H, rH) < tol("bf16")
     assert rel_l2(s, rs) < tol("bf16")
-    # state only: the same state, no output written
+    # state only: no output; the sequence may be split into segments whose
+    # partial states are summed, so only the rounding order differs
     none, H2, s2 = run(q, k, v, output=False)
-    assert none is None and torch.equal(H2, H) and torch.equal(s2, s)
+    assert none is None
+    assert rel_l2(H2, H.double().cpu().numpy()) < 1e-5
+    assert rel_l2(s2, s.double().cpu().numpy()) < 1e-5
+    assert rel_l2(H2, rH) < tol("bf16") and rel_l2(s2, rs) < tol("bf16")
 
 
 @pytest.mark.parametrize("d,T", [(32, 512), (64, 1024), (64, 768)])
@@ -86,3 +90,23 @@ def test_causality_of_the_tensor_core_path():
     o1, _, _ = run(q, k2, v2)
     assert torch.equal(o0[:, :, :t], o1[:, :, :t])
     assert not torch.equal(o0[:, :, t:], o1[:, :, t:])
+
+
+# final state only, over few heads: the state pass splits the sequence into
+# segments (grid z) and sums their partial states; with an initial state (the
+# first segment starts from it) and H_out aliasing H_in
+@pytest.mark.parametrize("d,T,H", [(32, 1024, 1), (32, 2048, 3), (64, 1024, 2), (64, 640, 1)])
+def test_segmented_state_pass(d, T, H):
+    q, k, v = prefill_inputs(1, H, T, d, dtype="bf16", seed=90 + d + T + H)
+    n0 = kata.launch_count()
+    none, Hs, ss = run(q, k, v, output=False)
+    assert none is None
+    assert kata.launch_count() - n0 == 3  # state pass + the two sums
+    _, rH, rs = oracle.recurrent(q, k, v, 1e-6, readout=False)
+    assert rel_l2(Hs, rH) < tol("bf16") and rel_l2(ss, rs) < tol("bf16")
+    # continue from it in place, state only again
+    q2, k2, v2 = prefill_inputs(1, H, T, d, dtype="bf16", seed=91 + d + T + H)
+    _, Hc, sc = run(q2, k2, v2, output=False, H_in=Hs, s_in=ss, H_out=Hs, s_out=ss)
+    qq, kk, vv = (torch.cat(x, dim=2) for x in ((q, q2), (k, k2), (v, v2)))
+    _, rH2, rs2 = oracle.recurrent(qq, kk, vv, 1e-6, readout=False)
+    assert rel_l2(Hc, rH2) < tol("bf16") and rel_l2(sc, rs2) < tol("bf16")
