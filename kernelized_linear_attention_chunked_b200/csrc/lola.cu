@@ -54,6 +54,26 @@ size_t partial_floats(int nh, int n, int d) {
 // Register-blocked scoring: each thread owns kCB candidates x kEB output
 // columns; the state slice streams through shared memory kRC rows at a time
 // and phi of those rows is built once per chunk for all the CTA's candidates.
+// Asynchronous global -> shared copies (16 or 4 bytes), grouped per commit.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 constexpr int kRC = 32;  // state rows per chunk
 constexpr int kCB = 4;   // candidates per thread
 constexpr int kEB = 16;  // output columns per thread
@@ -69,7 +89,9 @@ int partial_pass(int d, int n, int zsplit) {
 
 size_t state_partial_smem(int d, int pass) {
     const int D = packed_dim(d);
-    return ((size_t)pass * (d + 1) + (size_t)kRC * pass + (size_t)kRC * d + kRC) * sizeof(float) +
+    // candidates, phi of a chunk, two state chunks (H rows and s)
+    return ((size_t)pass * (d + 1) + (size_t)kRC * pass + 2 * ((size_t)kRC * d + kRC)) *
+               sizeof(float) +
            align_up((size_t)D * sizeof(uint16_t), 16);
 }
 
@@ -95,9 +117,9 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
     extern __shared__ float4 smem4[];
     float *Xs = reinterpret_cast<float *>(smem4);  // [pass][DH+1]
     float *Ph = Xs + (size_t)pass * (DH + 1);       // [kRC][pass]
-    float *Hc = Ph + (size_t)kRC * pass;            // [kRC][DH]
-    float *sc = Hc + kRC * DH;                      // [kRC]
-    uint16_t *tab = reinterpret_cast<uint16_t *>(sc + kRC);
+    float *Hc = Ph + (size_t)kRC * pass;            // [2][kRC][DH]: chunk k in buffer k % 2
+    float *sc = Hc + 2 * kRC * DH;                  // [2][kRC]
+    uint16_t *tab = reinterpret_cast<uint16_t *>(sc + 2 * kRC);
 
     build_pair_table(tab, DH);
     const Tin *Xh = X + (size_t)h * x_head_stride;
@@ -120,13 +142,28 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
 #pragma unroll
             for (int e = 0; e < kEB; ++e) acc[c][e] = 0.f;
         }
-        for (int rc = r0; rc < r1; rc += kRC) {
-            const int nr = min(kRC, r1 - rc);
-            __syncthreads();  // Xs written; the previous chunk's readers are done
+        // the slice streams through two shared-memory chunk buffers: the copy
+        // of chunk k + 1 is in flight while chunk k's phi is built and used
+        const int nchunk = (r1 - r0 + kRC - 1) / kRC;
+        auto issue = [&](int k) {
+            const int rc = r0 + k * kRC, nr = min(kRC, r1 - rc);
+            float *hb = Hc + (k & 1) * kRC * DH;
+            float *sb = sc + (k & 1) * kRC;
             for (int idx = tid; idx < nr * DH / 4; idx += kThreads)
-                reinterpret_cast<float4 *>(Hc)[idx] =
-                    reinterpret_cast<const float4 *>(Hh + (size_t)rc * DH)[idx];
-            for (int idx = tid; idx < nr; idx += kThreads) sc[idx] = sh[rc + idx];
+                cp_async16(hb + 4 * idx, Hh + (size_t)rc * DH + 4 * idx);
+            for (int idx = tid; idx < nr; idx += kThreads) cp_async4(sb + idx, sh + rc + idx);
+            cp_async_commit();
+        };
+        if (nchunk > 0) issue(0);
+        for (int k = 0; k < nchunk; ++k) {
+            const int rc = r0 + k * kRC, nr = min(kRC, r1 - rc);
+            const float *hb = Hc + (k & 1) * kRC * DH;
+            const float *sb = sc + (k & 1) * kRC;
+            cp_async_wait_all();  // this thread's copies of chunk k have landed
+            // every copy of chunk k is visible; every thread is done with chunk
+            // k - 1 (its buffer and Ph), and Xs is written
+            __syncthreads();
+            if (k + 1 < nchunk) issue(k + 1);
             for (int idx = tid; idx < nr * pass; idx += kThreads) {
                 const int rr = idx / pass, i = idx % pass;
                 Ph[rr * pass + i] = phi_entry(Xs + i * (DH + 1), tab[rc + rr]);
@@ -138,7 +175,7 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                     const float pv[kCB] = {ph.x, ph.y, ph.z, ph.w};
                     // columns 4 (q NEB + ej) .. +3: neighbouring threads read
                     // neighbouring 16-byte chunks (no bank conflicts)
-                    const float4 *hv = reinterpret_cast<const float4 *>(Hc + rr * DH);
+                    const float4 *hv = reinterpret_cast<const float4 *>(hb + rr * DH);
 #pragma unroll
                     for (int q = 0; q < kEB / 4; ++q) {
                         const float4 hq = hv[q * NEB + ej];
@@ -151,7 +188,7 @@ state_partial_kernel(const Tin *__restrict__ X, long x_head_stride, int n,
                         }
                     }
                     if (ej == 0) {
-                        const float sr = sc[rr];
+                        const float sr = sb[rr];
 #pragma unroll
                         for (int c = 0; c < kCB; ++c) den[c] = fmaf(pv[c], sr, den[c]);
                     }
