@@ -48,6 +48,17 @@ def test_status_strings_and_helpers():
         assert kata.packed_dim(d) == d * (d + 1) // 2
 
 
+def test_workspace_holds_segment_partial_states():
+    # a final-state-only bf16 call of one head over two 128-token chunks splits
+    # the sequence in two segments: their partial states must fit
+    L = kata.lib()
+    d, D = 32, 32 * 33 // 2
+    align = lambda x: (x + 255) // 256 * 256
+    parts = align(2 * D * d * 4) + align(2 * D * 4)
+    s_copy = align(D * 4)
+    assert L.kata_prefill_workspace_bytes(1, 1, 256, d, 64, 1) >= s_copy + parts
+
+
 def test_workspace_queries():
     L = kata.lib()
     assert L.kata_prefill_workspace_bytes(1, 1, 256, 16, 64, 0) > 0
