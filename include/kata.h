@@ -138,8 +138,12 @@ enum { KATA_FORM_AUTO = 0, KATA_FORM_CHUNKED = 1, KATA_FORM_QUADRATIC = 2 };
  *                        state is computed by the chunked form's state pass
  *                        at the same time, on a second stream the library
  *                        forks from `stream` and joins back to it with events
- *                        (one per device, shared by the calling threads).
- *                        workspace is not used (may be NULL, ws_bytes 0).
+ *                        (one per device, shared by the calling threads; a
+ *                        call made while `stream` is being captured into a
+ *                        CUDA graph brings the side stream into the capture,
+ *                        so no other thread may use this form on the same
+ *                        device during the capture). workspace is not used
+ *                        (may be NULL, ws_bytes 0).
  *   KATA_FORM_AUTO       what kata_prefill does: the quadratic form for a call
  *                        without H_in and H_out when it applies and
  *                        T <= kata_quadratic_max_tokens(d), the chunked form
