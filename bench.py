@@ -146,7 +146,8 @@ class ClockSampler:
 
 def traffic_record(kernel: str, workload: str):
     """ncu dram bytes per launch recorded under profiles/, if the kernel source
-    has not changed since the counters were taken (else None)."""
+    has not changed since the counters were taken (else None). The figure is
+    a recorded ncu measurement, not one taken by this run."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
@@ -159,28 +160,85 @@ def traffic_record(kernel: str, workload: str):
     return rec["bytes_per_launch"]
 
 
+def traffic_source(kernel: str, workload: str) -> str:
+    rec = None
+    p = ROOT / "profiles" / "traffic.json"
+    if p.exists():
+        rec = json.loads(p.read_text()).get(f"{kernel}@{workload}")
+    if traffic_record(kernel, workload) is None:
+        return "none: no ncu record for the current kernel source"
+    return (f"recorded: ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, "
+            f"{rec.get('case', workload)}, kernel source sha {rec['sha']}")
+
+
+def roofline(seconds: float, flops: float | None, nbytes: float | None, peaks,
+             tensor_key: str = "bf16_tflops") -> dict:
+    """Roofline of one launch or call that does `flops` algorithmic flops and
+    moves `nbytes` algorithmic bytes in `seconds`. The bound is the resource
+    whose floor time (work / measured peak) is the larger; both fractions are
+    given, each against its measured peak."""
+    out = {}
+    floors = {}
+    if flops:
+        pk = peaks[tensor_key]
+        out["tensor"] = {"achieved": flops / seconds / 1e12, "peak": pk, "unit": "TFLOP/s",
+                         "frac": flops / seconds / 1e12 / pk, "peak_key": tensor_key}
+        floors["tensor"] = flops / (pk * 1e12)
+    if nbytes:
+        pk = peaks["hbm_gbs"]
+        out["hbm"] = {"achieved": nbytes / seconds / 1e9, "peak": pk, "unit": "GB/s",
+                      "frac": nbytes / seconds / 1e9 / pk, "peak_key": "hbm_gbs"}
+        floors["hbm"] = nbytes / (pk * 1e9)
+    bound = max(floors, key=floors.get)
+    main = out[bound]
+    return {"bound": bound, "achieved": main["achieved"], "peak": main["peak"],
+            "unit": main["unit"], "frac": main["frac"], "seconds": seconds,
+            "floor_seconds": floors[bound], "algorithmic_flops": flops,
+            "algorithmic_bytes": nbytes, **out}
+
+
 # ---------------------------------------------------------------- oracle ----
 
-def cpu_baseline(w, max_heads: int | None = None, min_seconds: float = 0.0):
+def cpu_model() -> str:
+    try:
+        for line in Path("/proc/cpuinfo").read_text().splitlines():
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(w, max_heads: int | None = None, min_seconds: float = 0.0,
+                 threads: int | None = None):
     """The fp64 oracle (recurrent form, the fastest exact CPU form) on a
     bounded sample of the workload, scaled to tokens/s. The sample is
     `max_heads` heads of the workload (all by default), repeated until
-    `min_seconds` of CPU time have passed."""
+    `min_seconds` of CPU time have passed, on `threads` OpenMP threads (the
+    host's default when None; the heads are the parallel loop)."""
     import oracle
     q, k, v = prefill_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed, recipe=w.recipe)
     nh = w.B * w.H if max_heads is None else min(max_heads, w.B * w.H)
     qf, kf, vf = (x.reshape(w.B * w.H, w.T, w.d)[:nh] for x in (q, k, v))
-    reps, dt = 0, 0.0
-    t0 = time.perf_counter()
-    while reps == 0 or dt < min_seconds:
-        oracle.recurrent(qf, kf, vf, w.eps)
-        reps += 1
-        dt = time.perf_counter() - t0
+    default = oracle.threads()
+    if threads is not None:
+        oracle.set_threads(threads)
+    used = min(oracle.threads(), nh)  # one head per thread at a time
+    try:
+        reps, dt = 0, 0.0
+        t0 = time.perf_counter()
+        while reps == 0 or dt < min_seconds:
+            oracle.recurrent(qf, kf, vf, w.eps)
+            reps += 1
+            dt = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(default)
     tokens = reps * w.T * nh / w.H  # a token is one position of one sequence (all heads)
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"recurrent fp64 form, {nh} of {w.B * w.H} heads x {w.T} tokens, "
-                      f"{reps} repetition(s), {dt:.1f} s", "seconds": dt / reps}
+                      f"{reps} repetition(s), {dt:.1f} s, {used} thread(s)",
+            "seconds": dt / reps}
 
 
 def run_reference(args, rank: int):
@@ -188,12 +246,13 @@ def run_reference(args, rank: int):
         return
     import oracle  # noqa: F401
     w = WORKLOADS[HEADLINE]
-    nh = 8  # a bounded sample per step: 8 of 32 heads
+    # every step is the whole workload: all 32 heads x 2048 tokens (about 0.1 s
+    # on 16 host cores; the heads are the parallel loop)
     for _ in range(args.warmup):
-        cpu_baseline(w, max_heads=nh)
+        cpu_baseline(w)
     times, vals = [], []
     for _ in range(args.steps):
-        r = cpu_baseline(w, max_heads=nh)
+        r = cpu_baseline(w)
         times.append(r["seconds"])
         vals.append(r["value"])
     value = float(np.mean(vals))
@@ -204,7 +263,8 @@ def run_reference(args, rank: int):
             "config": {"workload": HEADLINE, "global_batch": w.B, "seq_len": w.T, "heads": w.H,
                        "head_dim": w.d, "chunk": w.chunk, "parallelism": "host cores"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle",
-                             "cores": r["cores"], "sample": r["sample"]},
+                             "cores": r["cores"], "cpu_model": r["cpu_model"],
+                             "sample": r["sample"]},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -285,7 +345,7 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
         fn = {"decode": lambda: bench_decode(kata, args, dev, stream, peaks, dist_on, world),
               "long_prefill": lambda: bench_long_prefill(kata, args, dev, stream, peaks,
                                                          dist_on, world),
-              "lola": lambda: bench_lola(kata, args, dev, stream, dist_on, world),
+              "lola": lambda: bench_lola(kata, args, dev, stream, peaks, dist_on, world),
               "sre_stress": lambda: bench_sre_stress(kata, args, dev, stream, peaks, dist_on,
                                                      world)}[args.only]
         res = fn()
@@ -298,6 +358,9 @@ def run_kata(args, rank: int, world: int, dist_on: bool):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(WORKLOADS[HEADLINE], min_seconds=10.0)
         cpu.pop("seconds")
+        # the same form on one thread: 2 heads (one thread walks the heads in turn)
+        one = cpu_baseline(WORKLOADS[HEADLINE], max_heads=2, min_seconds=3.0, threads=1)
+        cpu["one_thread"] = {"value": one["value"], "unit": "tokens/s", "sample": one["sample"]}
         line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -341,42 +404,29 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     form = kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16)
     path = "tc" if kata.prefill_uses_tensor_cores(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16) \
         else "simt"
-    flops = quadratic_flops(w) if form == "quadratic" else prefill_flops(w)
+    # the method's algorithmic flops (the chunked form's count, whichever form
+    # runs: the T^2 pair work the quadratic form does instead is not counted)
+    flops = prefill_flops(w)
     tflops = flops / (ms_step / 1e3) / 1e12
     lat = per_launch_ms(step, max(args.steps, 10), stream)
-    chunked = None
-    if form == "quadratic":
-        # one launch per call: the quadratic-form kernel
-        roof = {"bound": "tensor", "achieved": flops / (lat / 1e3) / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        kernel, dom_ms, kernels = "quad_kernel", lat, None
-        chunked = bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks)
-    elif path == "tc":
-        # the chunked form's two launches (state kernel, readout kernel) as one
-        roof = {"bound": "tensor", "achieved": flops / (lat / 1e3) / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        kernel, dom_ms = "state_kernel", lat
-        kernels = {"state_pass": state_pass(kata, w, sets, R, ws, args, stream, dev)}
-    else:
-        # fp32 FMA pipes: 148 SMs x 128 lanes x 2 flops x max SM clock
-        alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        roof = {"bound": "alu", "achieved": flops / (lat / 1e3) / 1e12, "peak": alu_peak,
-                "unit": "TFLOP/s"}
-        kernel, dom_ms, kernels = "prefill_simt_kernel", lat, None
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" \
-        else "fallback"
+    kernel = {"quadratic": "quad_kernel"}.get(form, "state_kernel+readout_kernel"
+                                               if path == "tc" else "prefill_simt_kernel")
+    # one launch per call for the quadratic form (the call time is that
+    # kernel's launch time); the chunked form's two launches are one call
+    roof = roofline(lat / 1e3, flops, prefill_bytes(w), peaks)
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json, burst)" \
+        if peak_kind == "measured" else "fallback"
     roof["kernel"] = kernel
-    roof["launch_ms"] = dom_ms
-    roof["algorithmic_flops"] = flops if kernel in ("quad_kernel", "prefill_simt_kernel") \
-        else None
+    roof["launch_ms"] = lat
     roof["traffic"] = traffic_record(kernel, HEADLINE)
-    roof["call_ms"] = lat
-    roof["call_tflops"] = flops / (lat / 1e3) / 1e12
-    roof["algorithmic_bytes"] = prefill_bytes(w)
-    roof["call_hbm_frac"] = prefill_bytes(w) / (lat / 1e3) / 1e9 / peaks["hbm_gbs"]
-    if kernels:
-        roof["kernels"] = kernels
+    roof["traffic_source"] = traffic_source(kernel, HEADLINE)
+    roof["counting"] = ("algorithmic flops per head-token 4D(d+1) + (C+1)(2d+1) "
+                        "(the chunked form's count); bytes q, k, v in + fp32 o out")
+    if form == "quadratic":
+        roof["executed_flops_quadratic_form"] = quadratic_flops(w)
+    chunked = bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks) \
+        if form == "quadratic" else None
+    with_state = bench_with_state(kata, w, sets, R, ws, args, stream, dev, peaks)
 
     # end to end: host q, k, v in, host o out, through the C ABI
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
@@ -401,7 +451,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
     if not args.headline_only:
         sub["decode"] = bench_decode(kata, args, dev, stream, peaks, dist_on, world)
         sub["long_prefill"] = bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world)
-        sub["lola"] = bench_lola(kata, args, dev, stream, dist_on, world)
+        sub["lola"] = bench_lola(kata, args, dev, stream, peaks, dist_on, world)
         sub["sre_stress"] = bench_sre_stress(kata, args, dev, stream, peaks, dist_on, world)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -417,6 +467,7 @@ def run_all(kata, args, rank, world, dist_on, dev, stream, peaks, peak_kind):
                         "frac_bf16_peak": tflops / peaks["bf16_tflops"],
                         "peak_source": peak_kind},
             "chunked_form": chunked,
+            "prefill_with_state": with_state,
             "roofline": roof, "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches,
             "wall_s": wall}
     line.update(sub)
@@ -463,12 +514,36 @@ def bench_chunked_form(kata, w, sets, R, ws, args, stream, dev, peaks):
     kata.sync_status()
     flops = prefill_flops(w)
     return {"ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
-            "flops_per_step": flops, "tflops": flops / (ms / 1e3) / 1e12,
-            "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-            "call_ms": lat,
+            "flops_per_step": flops, "call_ms": lat,
+            "roofline": roofline(lat / 1e3, flops, prefill_bytes(w), peaks),
             "traffic": {"state_kernel": traffic_record("state_kernel", HEADLINE),
                         "readout_kernel": traffic_record("readout_kernel", HEADLINE)},
             "state_only_call": state_pass(kata, w, sets, R, ws, args, stream, dev)}
+
+
+def bench_with_state(kata, w, sets, R, ws, args, stream, dev, peaks):
+    """The call a prefill that hands its state to decode makes: o and the final
+    state (H, s) of the same batch; kata_prefill takes the chunked form."""
+    outs = [torch.empty(w.B, w.H, w.T, w.d, device=dev) for _ in range(R)]
+    Hs = torch.empty(w.B, w.H, w.D, w.d, device=dev)
+    ss = torch.empty(w.B, w.H, w.D, device=dev)
+
+    def step(i):
+        qq, kk, vv = sets[i % R]
+        kata.prefill(qq, kk, vv, chunk=w.chunk, eps=w.eps, o=outs[i % R], H_out=Hs, s_out=ss,
+                     workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    ms = time_events(step, args.steps, stream) / args.steps
+    lat = per_launch_ms(step, max(args.steps, 10), stream)
+    kata.sync_status()
+    flops = prefill_flops(w)
+    # the final state (fp32 H and s) is written once on top of q, k, v, o
+    nbytes = prefill_bytes(w) + w.B * w.H * w.D * (w.d + 1) * 4
+    return {"form": kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16, True),
+            "ms_per_step": ms, "tokens_per_s": w.B * w.T / (ms / 1e3), "call_ms": lat,
+            "roofline": roofline(lat / 1e3, flops, nbytes, peaks)}
 
 
 def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
@@ -499,10 +574,13 @@ def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
     launches = kata.launch_count() - n0
     kata.sync_status()
     ms_step = ms / nsteps
-    gbs = decode_bytes(w) / (ms_step / 1e3) / 1e9
+    # per step and head: phi(k) v^T update and phi(q)^T [H | s] readout, 2 flops
+    # per multiply-add each, over the D (d+1) state entries
+    flops = float(w.B * w.H * 4 * D * (w.d + 1))
     return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B, nsteps, ms),
-            "us_per_step": 1e3 * ms_step, "steps": nsteps, "gbs": gbs,
-            "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_step": decode_bytes(w),
+            "us_per_step": 1e3 * ms_step, "steps": nsteps,
+            "roofline": roofline(ms_step / 1e3, flops, decode_bytes(w), peaks),
+            "bytes_per_step": decode_bytes(w),
             "gpu_launches": launches, "l2": "state 554 MB > 126 MB L2"}
 
 
@@ -534,17 +612,15 @@ def bench_sre_stress(kata, args, dev, stream, peaks, dist_on, world):
     ms = max_over_ranks(time_events(step, iters, stream), dist_on) / iters
     launches = (kata.launch_count() - n0) // iters
     kata.sync_status()
-    gbs = nbytes / (ms / 1e3) / 1e9
     # fp32 work: phi(k)^T [H | s] for every candidate, then a rank-one update
     # of [H | s] for every merged one (2 flops per multiply-add)
     flops = float(B * H * (n + (n - keep)) * D * (d + 1) * 2)
-    alu_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-    tflops = flops / (ms / 1e3) / 1e12
-    return {"workload": "sre_b64_h16_d64_n192_keep128", "ms_per_pass": ms, "gbs": gbs,
-            "frac_hbm": gbs / peaks["hbm_gbs"], "bytes_per_pass": nbytes,
-            "tflops_fp32": tflops, "frac_alu": tflops / alu_peak, "flops_per_pass": flops,
-            "bound": "alu (96 flop per state byte in fp32: SRE decides the kept set, so "
-                     "it stays fp32 on the CUDA cores)",
+    roof = roofline(ms / 1e3, None, nbytes, peaks)
+    roof["note"] = ("HBM roofline of the algorithmic bytes; the scores are fp32 "
+                    "(fp32_tflops gives the arithmetic rate, not a roofline)")
+    return {"workload": "sre_b64_h16_d64_n192_keep128", "ms_per_pass": ms,
+            "roofline": roof, "bytes_per_pass": nbytes,
+            "fp32_tflops": flops / (ms / 1e3) / 1e12, "flops_per_pass": flops,
             "gpu_launches_per_pass": launches, "l2": "state 554 MB > 126 MB L2"}
 
 
@@ -567,11 +643,12 @@ def bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world):
     kata.sync_status()
     fl = prefill_flops(w)
     return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B * w.T, 1, ms), "ms": ms,
-            "tflops": fl / (ms / 1e3) / 1e12, "frac_bf16_peak": fl / (ms / 1e3) / 1e12 /
-            peaks["bf16_tflops"], "l2": "inputs 335 MB > 126 MB L2"}
+            "form": kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16),
+            "roofline": roofline(ms / 1e3, fl, prefill_bytes(w), peaks),
+            "l2": "inputs 335 MB > 126 MB L2"}
 
 
-def bench_lola(kata, args, dev, stream, dist_on, world):
+def bench_lola(kata, args, dev, stream, peaks, dist_on, world):
     w = WORKLOADS["lola_b2_h8_t8192_d64"]
     q, k, v = (x.to(dev) for x in recall_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed))
     D = w.D
@@ -594,8 +671,16 @@ def bench_lola(kata, args, dev, stream, dist_on, world):
     ms = max_over_ranks(time_events(step, n, stream), dist_on) / n
     launches = (kata.launch_count() - n0) // n
     kata.sync_status()
+    # labelled state-streaming model: every update of every head reads and
+    # writes that head's fp32 state once (2 x D (d+1) x 4 bytes)
+    updates = w.T // w.window - 1
+    stream_bytes = float(2 * w.D * (w.d + 1) * 4 * updates * w.B * w.H)
+    roof = roofline(ms / 1e3, None, stream_bytes, peaks)
+    roof["model"] = ("state-streaming model: each of the 127 updates of each head reads and "
+                     "writes its 540,800-byte fp32 state once; the state fits in L2, so this "
+                     "is a yardstick, not the bytes HBM moves")
     return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
-            "updates": w.T // w.window - 1, "gpu_launches_per_pass": launches,
+            "updates": updates, "gpu_launches_per_pass": launches, "roofline": roof,
             "note": "includes two state zero-fills per pass (torch memset)"}
 
 

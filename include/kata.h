@@ -121,6 +121,22 @@ KATA_API int kata_prefill(const void *q, const void *k, const void *v, int dtype
  * cores, 0 = CUDA cores, -1 = invalid or unsupported arguments. */
 KATA_API int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype);
 
+/*
+ * Test hook for failure detection (no counterpart on the pages). Runs the
+ * quadratic form of kata_prefill (bf16 q, k, v [B, H, T, d], d = 32 or 64,
+ * T a multiple of 128, zero initial state) with one deliberate fault: in
+ * every CTA, the warp that issues the P [V | 1] MMAs first waits on a barrier
+ * that nothing ever arrives at, giving up after `polls` polls (1 .. 2^20).
+ * The CTA then takes its error path: every role stops waiting, drains the
+ * copies and MMAs it issued, frees its tensor memory and exits; o is not
+ * valid. The next kata_sync_status() on this device returns
+ * KATA_ERR_TIMEOUT with the site code 0x6FF (kata_last_error()), and the
+ * context stays usable for the calls that follow.
+ */
+KATA_API int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B, int H,
+                                      int T, int d, float eps, float *o, unsigned int polls,
+                                      void *stream);
+
 /* The two exact forms of a prefill. */
 enum { KATA_FORM_AUTO = 0, KATA_FORM_CHUNKED = 1, KATA_FORM_QUADRATIC = 2 };
 

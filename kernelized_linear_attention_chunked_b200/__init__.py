@@ -28,4 +28,5 @@ from ._binding import (  # noqa: F401
     quadratic_max_tokens,
     sre_score_topk,
     sync_status,
+    test_forced_timeout,
 )

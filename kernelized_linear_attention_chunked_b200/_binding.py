@@ -32,6 +32,7 @@ SIGNATURES = {
     "kata_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
                           _vp, _sz, _vp]),
     "kata_prefill_path": (_i, [_i, _i, _i, _i, _i, _i]),
+    "kata_test_forced_timeout": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, C.c_uint, _vp]),
     "kata_prefill_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
                              _vp, _sz, _vp, _i]),
     "kata_quadratic_max_tokens": (_i, [_i]),
@@ -152,6 +153,18 @@ def prefill(q, k, v, chunk: int, eps: float = 1e-6, H_in=None, s_in=None, state:
         _ptr(s_in), _ptr(o), _ptr(H_out), _ptr(s_out), workspace.data_ptr(), workspace.numel(),
         _stream(stream), FORMS[form]))
     return o, H_out, s_out
+
+
+def test_forced_timeout(q, k, v, polls: int, eps: float = 1e-6, o=None, stream=None):
+    """kata_test_forced_timeout: the quadratic form with a wait that nothing
+    completes (a failure-detection test hook). Returns o (not valid)."""
+    _dev(q, k, v)
+    B, Hh, T, d = q.shape
+    if o is None:
+        o = torch.empty(B, Hh, T, d, dtype=torch.float32, device=q.device)
+    _check("kata_test_forced_timeout", lib().kata_test_forced_timeout(
+        _ptr(q), _ptr(k), _ptr(v), B, Hh, T, d, eps, _ptr(o), polls, _stream(stream)))
+    return o
 
 
 def prefill_auto_form(B, H, T, d, chunk, dtype, with_state: bool = False) -> str:

@@ -32,6 +32,16 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     return r;
 }
 
+// Split cluster barrier, first half: this CTA is running (no memory ordering).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+// Second half: every CTA of the cluster has arrived, so every CTA has started
+// and its shared memory may be written through distributed shared memory.
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+
 // All threads of every CTA of the cluster: release this CTA's shared-memory
 // writes, acquire the others'.
 __device__ __forceinline__ void cluster_sync() {
@@ -80,6 +90,10 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         pk[at] = (xs[1][a] * xs[1][b]) * w;
     }
     __syncthreads();
+    // announce that this CTA runs; the partner waits for it before writing into
+    // this CTA's shared memory (the wait comes after the streaming loop, so the
+    // barrier costs nothing on the loop)
+    cluster_arrive_relaxed();
 
     const int cg = tid % CG, rsub = tid / CG;
     const float4 vv = reinterpret_cast<const float4 *>(xs[2])[cg];
@@ -128,6 +142,7 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     if (lane < CG) red[warp][lane] = acc;
     if (lane == 0) zred[warp] = z;
     __syncthreads();
+    cluster_wait();  // both CTAs of the cluster have started
     float zt = 0.f, num = 0.f;
     if (tid < DH) {
         for (int w = 0; w < NW; ++w) {

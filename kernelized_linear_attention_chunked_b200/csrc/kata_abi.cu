@@ -30,17 +30,27 @@ int cuda_fail(cudaError_t e, const char *what) {
 
 __device__ unsigned int g_error_word;
 
-// Address of this device's error word (looked up once per device).
+// Per-device caches below cover device ordinals 0 .. kMaxDevices - 1.
+constexpr int kMaxDevices = 128;
+
+// Address of this device's error word (looked up once per device, with the
+// device current; the lookup is serialised across host threads).
 unsigned int *error_word() {
-    static unsigned int *addr[64] = {nullptr};
+    static std::atomic<unsigned int *> addr[kMaxDevices];
+    static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    unsigned int *a = addr[dev].load(std::memory_order_acquire);
+    if (a) return a;
+    std::lock_guard<std::mutex> lock(mu);
+    a = addr[dev].load(std::memory_order_relaxed);
+    if (!a) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<unsigned int *>(p);
+        a = static_cast<unsigned int *>(p);
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 
 std::atomic<unsigned long long> g_launches{0};
@@ -54,9 +64,9 @@ struct SideStream {
 };
 
 SideStream *side_stream() {
-    static SideStream sides[64];
+    static SideStream sides[kMaxDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     SideStream &sd = sides[dev];
     std::lock_guard<std::mutex> lock(sd.mu);
     if (!sd.stream) {
@@ -143,7 +153,7 @@ int kata_sync_status(void *stream) {
         unsigned int zero = 0;
         e = cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return cuda_fail(e, "clear error word");
-        return fail(KATA_ERR_TIMEOUT, "a kernel's bounded wait ran out (code %u)", h);
+        return fail(KATA_ERR_TIMEOUT, "a kernel's bounded wait ran out (code 0x%X)", h);
     }
     return KATA_OK;
 }
@@ -311,6 +321,29 @@ int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype) {
     a.d = d;
     a.chunk = chunk;
     return dtype == KATA_BF16 && kata::prefill_tc_supported(a) ? 1 : 0;
+}
+
+int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B, int H, int T,
+                             int d, float eps, float *o, unsigned int polls, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_prefill(KATA_BF16, B, H, T, d, 128);
+    if (st) return st;
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_REQUIRE_PTR(o);
+    if (!quadratic_applies(KATA_BF16, B, H, T, d, false))
+        return fail(KATA_ERR_UNSUPPORTED, "the forced timeout runs the quadratic form: d = 32 or "
+                                          "64, T a multiple of 128");
+    if (polls < 1 || polls > (1u << 20))
+        return fail(KATA_ERR_INVALID_ARG, "polls=%u must be in [1, 2^20]", polls);
+    unsigned int *err = error_word();
+    if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
+    kata::PrefillArgs a{q, k, v, KATA_BF16, B, H, T, d, 128, eps, nullptr, nullptr, o,
+                        nullptr, nullptr, nullptr, 0, err};
+    cudaError_t e = kata::quad_tc(a, static_cast<cudaStream_t>(stream), polls);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_test_forced_timeout launch");
+    return KATA_OK;
 }
 
 size_t kata_prefill_host_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype) {

@@ -30,8 +30,10 @@ cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream);
 // tcgen05 quadratic form: o only, from a zero state; H_in, H_out, ws are
 // ignored. quad_tc_shape_ok tells the sizes it takes (bf16, d = 32 or 64, T a
 // multiple of 128); the caller checks that q, k, v, o are 16-byte aligned.
+// `stall` > 0 is the forced-timeout test hook (the kernel's error path runs
+// after a wait of at most `stall` polls on a barrier nothing arrives at).
 bool quad_tc_shape_ok(int dtype, int B, int H, int T, int d);
-cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream);
+cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream, unsigned int stall = 0);
 
 cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
                         int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream);

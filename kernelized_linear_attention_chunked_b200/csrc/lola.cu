@@ -438,7 +438,11 @@ hybrid_finish_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         qv[c] = a < DH ? to_f32(q[hoff + (size_t)i * DH + a]) : 0.f;
         num[c] = 0.f;
     }
-    float den = 0.f;
+    // The softmax weights are taken relative to m = max(0, max_j tau q.k_j)
+    // (raised on the fly, rescaling what was summed so far), and the state
+    // terms and eps are scaled by exp(-m) to match: the same quotient, with no
+    // exp overflow however large tau q.k gets.
+    float den = 0.f, mx = 0.f;
     const int nw = i - w0 + 1;
     for (int jj = 0; jj < nw + nc; ++jj) {
         const Tin *kj, *vj;
@@ -457,7 +461,15 @@ hybrid_finish_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        const float w = expf(tau * dot);
+        const float t = tau * dot;
+        if (t > mx) {
+            const float r = expf(mx - t);
+            den *= r;
+#pragma unroll
+            for (int c = 0; c < PL; ++c) num[c] *= r;
+            mx = t;
+        }
+        const float w = expf(t - mx);
         den += w;
 #pragma unroll
         for (int c = 0; c < PL; ++c) {
@@ -465,16 +477,22 @@ hybrid_finish_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             if (a < DH) num[c] = fmaf(w, to_f32(vj[a]), num[c]);
         }
     }
+    float sden = 0.f, snum[PL];
+#pragma unroll
+    for (int c = 0; c < PL; ++c) snum[c] = 0.f;
     for (int p = 0; p < P; ++p) {
         const float *src = part + (((size_t)p * nh + h) * nq + r) * (DH + 1);
-        den += src[DH];
+        sden += src[DH];
 #pragma unroll
         for (int c = 0; c < PL; ++c) {
             const int a = lane + 32 * c;
-            if (a < DH) num[c] += src[a];
+            if (a < DH) snum[c] += src[a];
         }
     }
-    const float inv = 1.f / (den + eps);
+    const float sc = mx > 0.f ? expf(-mx) : 1.f;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) num[c] = fmaf(snum[c], sc, num[c]);
+    const float inv = 1.f / (fmaf(sden + eps, sc, den));
 #pragma unroll
     for (int c = 0; c < PL; ++c) {
         const int a = lane + 32 * c;
@@ -780,14 +798,15 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+constexpr int kMaxDevices = 128;  // device ordinals the address cache covers
 std::mutex g_noalloc_mutex;
-void *g_noalloc_addr[128] = {nullptr};
+void *g_noalloc_addr[kMaxDevices] = {nullptr};
 
 cudaError_t noalloc_scratch(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     if (!g_noalloc_addr[dev]) {
         void *p = nullptr;

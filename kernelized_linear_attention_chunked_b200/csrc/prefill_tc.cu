@@ -74,6 +74,11 @@ __device__ __forceinline__ void worker_sync() {
     asm volatile("bar.sync 1, %0;" ::"r"(kWorkers) : "memory");
 }
 
+// worker_sync that also tells every worker whether all of them are still fine
+// (a worker whose bounded wait ran out passes false; all then stop together,
+// so none is left waiting at a later worker barrier).
+__device__ __forceinline__ bool worker_vote(bool ok) { return bar_sync_and(1, kWorkers, ok); }
+
 // Element offset of 16-byte chunk `c` of row `r` in a tile with 128-byte rows
 // and the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw128_chunk(int r, int c) {
@@ -106,7 +111,8 @@ enum StateBar {
     kSbAFull = 12,   // NA: Phi(K)^T tile written to tensor memory (4 warp arrivals)
     kSbDone = 14,    // NA: the MMAs of the chunk that used this A slot completed
     kSbSnap = 16,    // the workers read the accumulators at an interval end
-    kSbCount = 17
+    kSbDrain = 17,   // 2: an issuer's MMAs completed (teardown)
+    kSbCount = 19
 };
 
 // Transposed K tile: row a holds k[t][a] for the 128 tokens of the chunk as
@@ -151,10 +157,12 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = blockIdx.x, head = blockIdx.y;
-    unsigned int *err = p.err;
+    const ErrCtx err{p.err, tmem_slot + 1};
     constexpr int kTmaWarp = 4 + NI;
 
     if (threadIdx.x == 0) {
+        tmem_slot[1] = 0u;  // the CTA's abort flag
+        for (int i = 0; i < 2; ++i) mbar_init(&bar[kSbDrain + i], 1);
         for (int i = 0; i < L::KR; ++i) {
             mbar_init(&bar[kSbKFull + i], 1);
             mbar_init(&bar[kSbKFree + i], 4);
@@ -224,15 +232,17 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 }
                 if (!moved) {
                     __nanosleep(32);
-                    if ((++idle & 1023u) == 0u && *((volatile unsigned int *)err) != 0u) break;
+                    if ((++idle & 1023u) == 0u && cta_aborted(err)) break;
                 }
             }
-            if (nk < nch || nv < nch) atomicCAS(err, 0u, 0x401u);
-            // no copy may still be in flight when the CTA exits
-            for (int c = nch - L::KR < 0 ? 0 : nch - L::KR; c < nch; ++c)
-                mbar_wait(&bar[kSbKFull + c % L::KR], (c / L::KR) & 1, err, 0x403);
-            for (int c = nch - 2 < 0 ? 0 : nch - 2; c < nch; ++c)
-                mbar_wait(&bar[kSbVFull + (c & 1)], (c >> 1) & 1, err, 0x404);
+            if (nk < nch || nv < nch) report_timeout(err, 0x401u);
+            // no copy may still be in flight when the CTA exits. A tile is only
+            // issued once the previous phase of its barrier completed, so the
+            // last tile issued on each barrier is the only one to wait for.
+            for (int c = nk - L::KR < 0 ? 0 : nk - L::KR; c < nk; ++c)
+                mbar_drain(&bar[kSbKFull + c % L::KR], (c / L::KR) & 1, err, 0x403);
+            for (int c = nv - 2 < 0 ? 0 : nv - 2; c < nv; ++c)
+                mbar_drain(&bar[kSbVFull + (c & 1)], (c >> 1) & 1, err, 0x404);
         }
     } else if (warp >= 4) {
         // ---------------- MMA issuer `ii`: K-steps ii, ii + NI, ... ----------------
@@ -243,11 +253,12 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             const uint32_t acc = tmem + L::acc_col(ii);
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1, sa = c % NA;
-                mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412);
-                mbar_wait(&bar[kSbAFull + sa], (c / NA) & 1, err, 0x410);
+                if (!mbar_wait(&bar[kSbVFull + s], (c >> 1) & 1, err, 0x412)) break;
+                if (!mbar_wait(&bar[kSbAFull + sa], (c / NA) & 1, err, 0x410)) break;
                 // the state at an interval end must be read before it moves on
-                if (c > 0 && c % p.cpi == 0)
-                    mbar_wait(&bar[kSbSnap], (c / p.cpi - 1) & 1, err, 0x411);
+                if (c > 0 && c % p.cpi == 0 &&
+                    !mbar_wait(&bar[kSbSnap], (c / p.cpi - 1) & 1, err, 0x411))
+                    break;
                 tc_fence_after();
                 const uint32_t v = smem_u32(sm + L::V0 + s * S::VBYTES);
 #pragma unroll
@@ -257,6 +268,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 mma_commit(&bar[kSbVFree + s]);
                 mma_commit(&bar[kSbDone + sa]);
             }
+            // every MMA this thread issued has completed before the teardown
+            mma_commit(&bar[kSbDrain + ii]);
+            mbar_drain(&bar[kSbDrain + ii], 0, err, 0x413);
         }
     } else {
         // ---------------- workers: one thread per feature row ----------------
@@ -313,9 +327,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
         // (row n < DH = column n of H, rows DH.. = s), then one bulk store
         // (thread 0 waits for the previous bulk store's read of the staging
         // buffer before the first worker sync of each chunk)
-        auto write_snapshot = [&](int g, const float (&x)[DH + 1]) {
-            if (p.snap == nullptr) return;
-            if (valid) {
+        auto write_snapshot = [&](int g, const float (&x)[DH + 1], bool ok) -> bool {
+            if (p.snap == nullptr) return ok;
+            if (ok && valid) {
                 uint8_t *row = stage + (f >> 6) * S::SLICE_BYTES;
                 const int fl = f & 63;
 #pragma unroll
@@ -326,13 +340,15 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                         __float2bfloat16_rn(n < DH ? x[n] : x[DH]);
             }
             fence_proxy_async_smem();
-            worker_sync();
+            if (!worker_vote(ok)) return false;
             if (f == 0)
                 bulk_store(p.snap + (((size_t)head * p.nint + g) * S::NS + 2 * tile) *
                                         S::SLICE_BYTES,
                            stage, nvalid * S::SLICE_BYTES);
+            return true;
         };
-        if (H_in) write_snapshot(0, init);
+        bool ok = true;  // warp-uniform: every wait of this warp so far succeeded
+        if (H_in) ok = write_snapshot(0, init, ok);
         if (f == 0) bulk_wait_read();
         // the state: sum of the issuers' accumulators, columns 0..DH-1 and s
         auto read_acc = [&](float (&x)[DH + 1]) {
@@ -355,11 +371,13 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
         };
 
         constexpr int NCB = DH / 8;  // 8-column blocks of a K row
+        // every worker reaches every worker_vote below (no worker leaves the
+        // loop on its own), so a failed wait never strands the others there
         for (int c = 0; c < nch; ++c) {
             const int sa = c % NA, ks = c % L::KR;
             // transpose the K tile in 8 x 8 blocks (8 tokens x 8 columns per thread)
-            warp_wait(&bar[kSbKFull + ks], (c / L::KR) & 1, err, 0x420);
-            if (f < 16 * NCB) {
+            ok = ok && warp_wait(&bar[kSbKFull + ks], (c / L::KR) & 1, err, 0x420);
+            if (ok && f < 16 * NCB) {
                 const uint8_t *kb = sm + L::K0 + ks * kTileBytes;
                 const int tb = f / NCB, cb = f % NCB;
                 uint32_t x[8][4];
@@ -383,9 +401,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kSbKFree + ks]);
+            if (ok && lane == 0) mbar_arrive(&bar[kSbKFree + ks]);
             if (f == 0) bulk_wait_read();  // staging buffer free for the next snapshot
-            worker_sync();  // K^T complete
+            if (!(ok = worker_vote(ok))) break;  // K^T complete
             // Phi(K)^T row of feature (ra, rb): 128 tokens, two per 32-bit column
             uint32_t a_row[64];
 #pragma unroll
@@ -399,9 +417,9 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             }
             worker_sync();  // K^T free for the next chunk
             // A slot sa was last read by chunk c - NA
-            if (c >= NA) warp_wait(&bar[kSbDone + sa], (c / NA - 1) & 1, err, 0x421);
+            if (c >= NA) ok = warp_wait(&bar[kSbDone + sa], (c / NA - 1) & 1, err, 0x421);
             tc_fence_after();
-            {
+            if (ok) {
                 uint32_t r[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -413,24 +431,24 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[kSbAFull + sa]);
+            if (ok && lane == 0) mbar_arrive(&bar[kSbAFull + sa]);
             // chunk c opens interval g: the state after chunk c - 1 is snapshot g
             // (A(c) is already published, so the issuers wait only for this read)
             if (c > 0 && c % p.cpi == 0) {
-                warp_wait(&bar[kSbDone + (c - 1) % NA], ((c - 1) / NA) & 1, err, 0x422);
+                if (ok) ok = warp_wait(&bar[kSbDone + (c - 1) % NA], ((c - 1) / NA) & 1, err, 0x422);
                 tc_fence_after();
                 float x[DH + 1];
-                read_acc(x);
+                if (ok) read_acc(x);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kSbSnap]);
-                write_snapshot(c / p.cpi, x);
+                if (ok && lane == 0) mbar_arrive(&bar[kSbSnap]);
+                ok = write_snapshot(c / p.cpi, x, ok);
             }
         }
         // final state, converted to the canonical layout
-        warp_wait(&bar[kSbDone + (nch - 1) % NA], ((nch - 1) / NA) & 1, err, 0x423);
+        if (ok) ok = warp_wait(&bar[kSbDone + (nch - 1) % NA], ((nch - 1) / NA) & 1, err, 0x423);
         tc_fence_after();
-        if (H_out) {
+        if (ok && H_out) {
             float fin[DH + 1];
             read_acc(fin);
             if (valid && ra <= rb) {
@@ -487,7 +505,8 @@ enum ReadBar {
     kRbPFree = kRbPFull + kRP,
     kRbAqFull = kRbPFree + kRP,  // 4 warp arrivals
     kRbAqFree = kRbAqFull + kRQMax,
-    kRbCount = kRbAqFree + kRQMax
+    kRbDrain = kRbAqFree + kRQMax,  // 2: an issuer's MMAs completed (teardown)
+    kRbCount = kRbDrain + 2
 };
 
 template <int DH, int NIR>
@@ -529,7 +548,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m = blockIdx.x, head = blockIdx.y;  // query tile, (batch, head)
-    unsigned int *err = p.err;
+    const ErrCtx err{p.err, tmem_slot + 1};
 
     const int g = m / p.cpi;               // snapshot interval of this query tile
     const int kt0 = g * p.cpi;             // first key tile of the interval
@@ -549,6 +568,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             const bool four = i == kRbSFree || (i >= kRbAqFull && i < kRbAqFull + kRQMax);
             mbar_init(&bar[i], four ? 4 : (i == kRbODone ? NIR : 1));
         }
+        tmem_slot[1] = 0u;  // the CTA's abort flag
         fence_barrier_init();
     }
     if (warp == 4) {
@@ -568,38 +588,46 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             prefetch_tensormap(&mq);
             prefetch_tensormap(&mk);
             prefetch_tensormap(&mv);
-            auto load_p = [&](int s) {
+            int nk = 0, nv = 0, np = 0;  // tiles and slices issued
+            auto load_p = [&](int s) -> bool {
                 const int slot = s % kRP;
-                if (s >= kRP) mbar_wait(&bar[kRbPFree + slot], ((s / kRP) - 1) & 1, err, 0x501);
+                if (s >= kRP && !mbar_wait(&bar[kRbPFree + slot], ((s / kRP) - 1) & 1, err, 0x501))
+                    return false;
                 mbar_arrive_expect_tx(&bar[kRbPFull + slot], S::SLICE_BYTES);
                 bulk_load(sm + L::P + slot * S::SLICE_BYTES, snap + (size_t)s * S::SLICE_BYTES,
                           S::SLICE_BYTES, &bar[kRbPFull + slot]);
+                ++np;
+                return true;
             };
-            auto load_kv = [&](int u) {
+            auto load_kv = [&](int u) -> bool {
                 const int y = (int)(row0 + (long)(kt0 + u) * kTile);
-                if (u > 0) mbar_wait(&bar[kRbKFree], (u - 1) & 1, err, 0x502);
+                if (u > 0 && !mbar_wait(&bar[kRbKFree], (u - 1) & 1, err, 0x502)) return false;
                 mbar_arrive_expect_tx(&bar[kRbKFull], kTileBytes);
                 tma_load_2d(sm + L::K, &mk, 0, y, &bar[kRbKFull]);
-                if (u > 0) mbar_wait(&bar[kRbVFree], (u - 1) & 1, err, 0x503);
+                ++nk;
+                if (u > 0 && !mbar_wait(&bar[kRbVFree], (u - 1) & 1, err, 0x503)) return false;
                 mbar_arrive_expect_tx(&bar[kRbVFull], S::VBYTES);
                 tma_load_2d(sm + L::V, &mv, 0, y, &bar[kRbVFull]);
+                ++nv;
+                return true;
             };
             mbar_arrive_expect_tx(&bar[kRbQFull], kTileBytes);
             tma_load_2d(sm + L::Q, &mq, 0, (int)(row0 + (long)m * kTile), &bar[kRbQFull]);
-            load_kv(0);
+            bool ok = load_kv(0);
             // the snapshots are written by the state kernel just before this one
-            if (n_inter > 0) grid_dependency_wait();
+            if (ok && n_inter > 0) grid_dependency_wait();
             const int first_p = n_inter < kRP ? n_inter : kRP;
-            for (int s = 0; s < first_p; ++s) load_p(s);
-            for (int u = 1; u < n_half / 2; ++u) load_kv(u);
-            for (int s = first_p; s < n_inter; ++s) load_p(s);
-            // no copy may still be in flight when the CTA exits
-            mbar_wait(&bar[kRbQFull], 0, err, 0x504);
-            const int nu = n_half / 2;
-            mbar_wait(&bar[kRbKFull], (nu - 1) & 1, err, 0x505);
-            mbar_wait(&bar[kRbVFull], (nu - 1) & 1, err, 0x506);
-            for (int s = n_inter - kRP < 0 ? 0 : n_inter - kRP; s < n_inter; ++s)
-                mbar_wait(&bar[kRbPFull + s % kRP], (s / kRP) & 1, err, 0x507);
+            for (int s = 0; ok && s < first_p; ++s) ok = load_p(s);
+            for (int u = 1; ok && u < n_half / 2; ++u) ok = load_kv(u);
+            for (int s = first_p; ok && s < n_inter; ++s) ok = load_p(s);
+            // no copy may still be in flight when the CTA exits. A copy is only
+            // issued once the previous phase of its barrier completed, so the
+            // last copy issued on each barrier is the only one to wait for.
+            mbar_drain(&bar[kRbQFull], 0, err, 0x504);
+            if (nk > 0) mbar_drain(&bar[kRbKFull], (nk - 1) & 1, err, 0x505);
+            if (nv > 0) mbar_drain(&bar[kRbVFull], (nv - 1) & 1, err, 0x506);
+            for (int s = np - kRP < 0 ? 0 : np - kRP; s < np; ++s)
+                mbar_drain(&bar[kRbPFull + s % kRP], (s / kRP) & 1, err, 0x507);
         }
     } else if (warp >= 4) {
         // ---------------- MMA issuer `ii` ----------------
@@ -611,9 +639,9 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             const uint32_t q_a = smem_u32(sm + L::Q), k_a = smem_u32(sm + L::K);
             const uint32_t v_a = smem_u32(sm + L::V), ones = smem_u32(sm + L::ONES);
             const uint32_t o_acc = tmem + L::o_col(ii);
-            auto issue_s = [&](int j) {  // S = Q K^T for 64-key half j
+            auto issue_s = [&](int j) -> bool {  // S = Q K^T for 64-key half j
                 const int u = j >> 1, h = j & 1;
-                if (h == 0) mbar_wait(&bar[kRbKFull], u & 1, err, 0x510);
+                if (h == 0 && !mbar_wait(&bar[kRbKFull], u & 1, err, 0x510)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk)
@@ -621,25 +649,28 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                            i_s, kk > 0);
                 mma_commit(&bar[kRbSFull]);
                 if (h == 1) mma_commit(&bar[kRbKFree]);
+                return true;
             };
-            if (ii == 0) {
-                mbar_wait(&bar[kRbQFull], 0, err, 0x511);
-                issue_s(0);
-            }
+            bool ok = true;
+            if (ii == 0) ok = mbar_wait(&bar[kRbQFull], 0, err, 0x511) && issue_s(0);
             int uses = 0;  // this issuer's items so far
-            for (int it = 0; it < n_items; ++it) {
+            for (int it = 0; ok && it < n_items; ++it) {
                 if (issuer_of(it) != ii) continue;
                 const int u = uses++;
                 const int slot = ii * SPI + u % SPI;
                 const uint32_t ph = (uint32_t)(u / SPI) & 1u;
                 if (it < n_half) {
                     const int j = it, h = j & 1;
-                    if (j + 1 < n_half) {
-                        mbar_wait(&bar[kRbSFree], j & 1, err, 0x512);
-                        issue_s(j + 1);
+                    if (j + 1 < n_half &&
+                        !(mbar_wait(&bar[kRbSFree], j & 1, err, 0x512) && issue_s(j + 1))) {
+                        ok = false;
+                        break;
                     }
-                    mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x513);
-                    if (h == 0) mbar_wait(&bar[kRbVFull], (j >> 1) & 1, err, 0x514);
+                    if (!mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x513) ||
+                        (h == 0 && !mbar_wait(&bar[kRbVFull], (j >> 1) & 1, err, 0x514))) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -649,8 +680,11 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                     if (h == 1) mma_commit(&bar[kRbVFree]);
                 } else {
                     const int s = it - n_half, ps = s % kRP;
-                    mbar_wait(&bar[kRbPFull + ps], (s / kRP) & 1, err, 0x516);
-                    mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x515);
+                    if (!mbar_wait(&bar[kRbPFull + ps], (s / kRP) & 1, err, 0x516) ||
+                        !mbar_wait(&bar[kRbAqFull + slot], ph, err, 0x515)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t pa = smem_u32(sm + L::P + ps * S::SLICE_BYTES);
 #pragma unroll
@@ -661,7 +695,10 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                     mma_commit(&bar[kRbPFree + ps]);
                 }
             }
-            mma_commit(&bar[kRbODone]);
+            if (ok) mma_commit(&bar[kRbODone]);
+            // every MMA this thread issued has completed before the teardown
+            mma_commit(&bar[kRbDrain + ii]);
+            mbar_drain(&bar[kRbDrain + ii], 0, err, 0x517);
         }
     } else {
         // ---------------- workers: one thread per query row ----------------
@@ -682,9 +719,9 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                 o4[x] = make_uint4(kOnesBf16x2, kOnesBf16x2, kOnesBf16x2, kOnesBf16x2);
             fence_proxy_async_smem();
         }
-        warp_wait(&bar[kRbQFull], 0, err, 0x520);
+        bool ok = warp_wait(&bar[kRbQFull], 0, err, 0x520);
         int uses0 = 0, uses1 = 0;  // items so far of issuer 0 and issuer 1
-        for (int it = 0; it < n_items; ++it) {
+        for (int it = 0; ok && it < n_items; ++it) {
             const int iss = issuer_of(it);
             const int u = iss == 0 ? uses0++ : uses1++;
             const int slot = iss * SPI + u % SPI;
@@ -693,7 +730,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                 // intra: squared scores of 64 keys, causal mask on the diagonal tile
                 const int j = it, h = j & 1, u = j >> 1;
                 const bool diag = kt0 + u == m;
-                warp_wait(&bar[kRbSFull], j & 1, err, 0x521);
+                if (!(ok = warp_wait(&bar[kRbSFull], j & 1, err, 0x521))) break;
                 tc_fence_after();
                 float sv[64];
 #pragma unroll
@@ -732,7 +769,8 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
                     for (int bb = 0; bb < 4; ++bb) pk[4 * a + bb] = hmul2(qa, wb[bb]);
                 }
             }
-            if (u >= SPI) warp_wait(&bar[kRbAqFree + slot], (u / SPI - 1) & 1, err, 0x522);
+            if (u >= SPI && !(ok = warp_wait(&bar[kRbAqFree + slot], (u / SPI - 1) & 1, err, 0x522)))
+                break;
             tc_fence_after();
             {
                 uint32_t r[16];
@@ -749,7 +787,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             if (lane == 0) mbar_arrive(&bar[kRbAqFull + slot]);
         }
         // epilogue: o = numerator / (denominator + eps), summed over the issuers
-        warp_wait(&bar[kRbODone], 0, err, 0x523);
+        if (ok) ok = warp_wait(&bar[kRbODone], 0, err, 0x523);
         tc_fence_after();
         float num[DH], den = 0.f;
 #pragma unroll
@@ -770,7 +808,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
         float4 *dst =
             reinterpret_cast<float4 *>(p.o + ((size_t)head * p.nch * kTile + (size_t)m * kTile + i) * DH);
 #pragma unroll
-        for (int n = 0; n < DH; n += 4)
+        for (int n = 0; ok && n < DH; n += 4)
             dst[n / 4] = make_float4(num[n] * inv, num[n + 1] * inv, num[n + 2] * inv,
                                      num[n + 3] * inv);
     }

@@ -37,6 +37,10 @@ struct QuadParams {
     float eps;
     float *o;
     unsigned int *err;
+    // test hook, 0 in every product call: the P [V | 1] issuer first waits at
+    // most `stall` polls on a barrier that nothing arrives at, so the CTA's
+    // bounded waits run out and it tears down through its error path
+    unsigned int stall;
 };
 
 enum QuadBar {
@@ -50,7 +54,10 @@ enum QuadBar {
     kQbPFull = 13,  // 2 P slots: the squared scores are written (4 warp arrivals)
     kQbPFree = 15,  // 2 P slots: the MMAs that read them completed
     kQbODone = 17,
-    kQbCount = 18
+    kQbSDrain = 18,  // the S issuer's MMAs completed (teardown)
+    kQbPDrain = 19,  // the P [V | 1] issuer's MMAs completed (teardown)
+    kQbNever = 20,   // nothing arrives here (the test hook's stall)
+    kQbCount = 21
 };
 
 // Square two fp32 scores (one packed f32x2 multiply, round to nearest) and
@@ -108,13 +115,14 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
     const int m = p.nch - 1 - (int)blockIdx.y;  // query tile: the longest rows launch first
     const int nh = 2 * (m + 1);                 // 64-key halves up to the diagonal
     const long row0 = (long)head * p.nch * kTile;
-    unsigned int *err = p.err;
+    const ErrCtx err{p.err, tmem_slot + 1};
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQbCount; ++i) {
             const bool four = (i >= kQbSFree && i < kQbSFree + 2) || (i >= kQbPFull && i < kQbPFull + 2);
             mbar_init(&bar[i], four ? 4 : 1);
         }
+        tmem_slot[1] = 0u;  // the CTA's abort flag
         fence_barrier_init();
     }
     if (warp == L::ISSUER_WARP) {
@@ -134,34 +142,39 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
             prefetch_tensormap(&mv);
             mbar_arrive_expect_tx(&bar[kQbQFull], kTileBytes);
             tma_load_2d(sm + L::Q, &mq, 0, (int)(row0 + (long)m * kTile), &bar[kQbQFull]);
+            int nk = 0, nv = 0;  // K and V tiles issued
             for (int u = 0; u <= m; ++u) {
                 const int st = u & 1;
                 const int y = (int)(row0 + (long)u * kTile);
-                if (u >= 2) mbar_wait(&bar[kQbKFree + st], ((u >> 1) - 1) & 1, err, 0x601);
+                if (u >= 2 && !mbar_wait(&bar[kQbKFree + st], ((u >> 1) - 1) & 1, err, 0x601)) break;
                 mbar_arrive_expect_tx(&bar[kQbKFull + st], kTileBytes);
                 tma_load_2d(sm + L::K0 + st * kTileBytes, &mk, 0, y, &bar[kQbKFull + st]);
-                if (u >= 2) mbar_wait(&bar[kQbVFree + st], ((u >> 1) - 1) & 1, err, 0x602);
+                ++nk;
+                if (u >= 2 && !mbar_wait(&bar[kQbVFree + st], ((u >> 1) - 1) & 1, err, 0x602)) break;
                 mbar_arrive_expect_tx(&bar[kQbVFull + st], S::VBYTES);
                 tma_load_2d(sm + L::V0 + st * S::VBYTES, &mv, 0, y, &bar[kQbVFull + st]);
+                ++nv;
             }
-            // no copy may still be in flight when the CTA exits
-            mbar_wait(&bar[kQbQFull], 0, err, 0x603);
-            for (int u = m - 1 < 0 ? 0 : m - 1; u <= m; ++u) {
-                mbar_wait(&bar[kQbKFull + (u & 1)], (u >> 1) & 1, err, 0x604);
-                mbar_wait(&bar[kQbVFull + (u & 1)], (u >> 1) & 1, err, 0x605);
-            }
+            // no copy may still be in flight when the CTA exits. A tile is only
+            // issued once the previous phase of its barrier completed, so the
+            // last tile issued on each barrier is the only one to wait for.
+            mbar_drain(&bar[kQbQFull], 0, err, 0x603);
+            for (int u = nk - 2 < 0 ? 0 : nk - 2; u < nk; ++u)
+                mbar_drain(&bar[kQbKFull + (u & 1)], (u >> 1) & 1, err, 0x604);
+            for (int u = nv - 2 < 0 ? 0 : nv - 2; u < nv; ++u)
+                mbar_drain(&bar[kQbVFull + (u & 1)], (u >> 1) & 1, err, 0x605);
         }
     } else if (warp == L::ISSUER_WARP) {
         // ---------------- S issuer: S = Q K^T for half j into buffer j % NSB ----------------
         if (lane == 0) {
             const uint32_t i_s = idesc_bf16(128, 64, 0, 0);
             const uint32_t q_a = smem_u32(sm + L::Q), k_a = smem_u32(sm + L::K0);
-            mbar_wait(&bar[kQbQFull], 0, err, 0x614);
-            for (int j = 0; j < nh; ++j) {
+            const bool ok = mbar_wait(&bar[kQbQFull], 0, err, 0x614);
+            for (int j = 0; ok && j < nh; ++j) {
                 const int u = j >> 1, h = j & 1, st = u & 1, b = j % NSB;
                 // the workers read this buffer's previous scores
-                if (j >= NSB) mbar_wait(&bar[kQbSFree + b], (j / NSB - 1) & 1, err, 0x610);
-                if (h == 0) mbar_wait(&bar[kQbKFull + st], (u >> 1) & 1, err, 0x611);
+                if (j >= NSB && !mbar_wait(&bar[kQbSFree + b], (j / NSB - 1) & 1, err, 0x610)) break;
+                if (h == 0 && !mbar_wait(&bar[kQbKFull + st], (u >> 1) & 1, err, 0x611)) break;
                 tc_fence_after();
                 const uint32_t kb = k_a + st * kTileBytes + h * 64 * 128;
 #pragma unroll
@@ -171,16 +184,21 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
                 mma_commit(&bar[kQbSFull + b]);
                 if (h == 1) mma_commit(&bar[kQbKFree + st]);
             }
+            // every MMA this thread issued has completed before the teardown
+            mma_commit(&bar[kQbSDrain]);
+            mbar_drain(&bar[kQbSDrain], 0, err, 0x615);
         }
     } else if (warp == L::PV_WARP) {
         // ---------------- P [V | 1] issuer: [N | Z] += P [V | 1] for half j ----------------
         if (lane == 0) {
             const uint32_t i_av = idesc_bf16(128, S::NACC, 0, 1);
             const uint32_t v_a = smem_u32(sm + L::V0), ones = smem_u32(sm + L::ONES);
-            for (int j = 0; j < nh; ++j) {
+            bool ok = p.stall == 0u || mbar_wait(&bar[kQbNever], 0, err, 0x6FF, p.stall);
+            for (int j = 0; ok && j < nh; ++j) {
                 const int u = j >> 1, h = j & 1, st = u & 1, ps = j % NP;
-                mbar_wait(&bar[kQbPFull + ps], (j / NP) & 1, err, 0x612);
-                if (h == 0) mbar_wait(&bar[kQbVFull + st], (u >> 1) & 1, err, 0x613);
+                ok = mbar_wait(&bar[kQbPFull + ps], (j / NP) & 1, err, 0x612) &&
+                     (h != 0 || mbar_wait(&bar[kQbVFull + st], (u >> 1) & 1, err, 0x613));
+                if (!ok) break;
                 tc_fence_after();
                 const uint32_t vb = v_a + st * S::VBYTES;
 #pragma unroll
@@ -190,7 +208,9 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
                 mma_commit(&bar[kQbPFree + ps]);
                 if (h == 1) mma_commit(&bar[kQbVFree + st]);
             }
-            mma_commit(&bar[kQbODone]);
+            if (ok) mma_commit(&bar[kQbODone]);
+            mma_commit(&bar[kQbPDrain]);
+            mbar_drain(&bar[kQbPDrain], 0, err, 0x616);
         }
     } else {
         // ---------------- workers: thread = query row = tensor-memory lane ----------------
@@ -198,10 +218,11 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         // the all-ones block; the first P-full arrival publishes it to the MMAs
         fill_ones(sm + L::ONES, i, kWorkers);
+        bool ok = true;
         for (int j = 0; j < nh; ++j) {
             const int h = j & 1, b = j % NSB, ps = j % NP;
             const bool diag = (j >> 1) == m;
-            warp_wait(&bar[kQbSFull + b], (j / NSB) & 1, err, 0x620);
+            if (!(ok = warp_wait(&bar[kQbSFull + b], (j / NSB) & 1, err, 0x620))) break;
             tc_fence_after();
             float sv[64];
 #pragma unroll
@@ -230,7 +251,8 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
                 for (int e = 0; e < 32; ++e)
                     pk[e] = sq_pack(__float_as_uint(sv[2 * e]), __float_as_uint(sv[2 * e + 1]));
             }
-            if (j >= NP) warp_wait(&bar[kQbPFree + ps], (j / NP - 1) & 1, err, 0x621);
+            if (j >= NP && !(ok = warp_wait(&bar[kQbPFree + ps], (j / NP - 1) & 1, err, 0x621)))
+                break;
             tc_fence_after();
             {
                 uint32_t r[16];
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
             if (lane == 0) mbar_arrive(&bar[kQbPFull + ps]);
         }
         // epilogue: o = N / (Z + eps)
-        warp_wait(&bar[kQbODone], 0, err, 0x622);
+        if (ok) ok = warp_wait(&bar[kQbODone], 0, err, 0x622);
         tc_fence_after();
         uint32_t r[DH / 16 + 1][16];
 #pragma unroll
@@ -256,7 +278,7 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
         const float inv = 1.f / (__uint_as_float(r[DH / 16][0]) + p.eps);
         float4 *dst = reinterpret_cast<float4 *>(p.o + (row0 + (long)m * kTile + i) * DH);
 #pragma unroll
-        for (int n = 0; n < DH; n += 4)
+        for (int n = 0; ok && n < DH; n += 4)
             dst[n / 4] = make_float4(__uint_as_float(r[n / 16][n % 16]) * inv,
                                      __uint_as_float(r[n / 16][n % 16 + 1]) * inv,
                                      __uint_as_float(r[n / 16][n % 16 + 2]) * inv,
@@ -272,13 +294,13 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
 }
 
 template <int DH>
-cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
+cudaError_t launch(const PrefillArgs &a, cudaStream_t stream, unsigned int stall) {
     using L = QuadCfg<DH>;
     const int nheads = a.B * a.H, nch = a.T / kTile;
     CUtensorMap mq, mk, mv;
     if (!make_qkv_maps(&mq, &mk, &mv, a.q, a.k, a.v, DH, (long)nheads * a.T))
         return cudaErrorInvalidValue;
-    QuadParams qp{nch, a.eps, a.o, a.err};
+    QuadParams qp{nch, a.eps, a.o, a.err, stall};
     cudaError_t e = set_smem_once<quad_kernel<DH>>(L::BYTES);
     if (e != cudaSuccess) return e;
     quad_kernel<DH><<<dim3(nheads, nch), L::THREADS, L::BYTES, stream>>>(mq, mk, mv, qp);
@@ -292,10 +314,10 @@ bool quad_tc_shape_ok(int dtype, int B, int H, int T, int d) {
            T / kTile <= 65535 && (long)B * H * T < (1L << 31) && (long)B * H <= 0x7FFFFFFFL;
 }
 
-cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream) {
+cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream, unsigned int stall) {
     if (!quad_tc_shape_ok(a.dtype, a.B, a.H, a.T, a.d) || a.o == nullptr)
         return cudaErrorNotSupported;
-    return a.d == 64 ? launch<64>(a, stream) : launch<32>(a, stream);
+    return a.d == 64 ? launch<64>(a, stream, stall) : launch<32>(a, stream, stall);
 }
 
 }  // namespace kata

@@ -54,18 +54,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Non-blocking probe of the phase with this parity (try_wait may suspend the
 // thread for a while; a thread that polls several barriers uses this).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
@@ -80,30 +68,66 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: returns false (and records `code` in *err) if the phase with
-// this parity has not completed after `limit` polls. A phase that has already
-// completed is seen by the cheap non-blocking probe; only a wait that has to
-// wait uses the suspending form.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
+// Where a CTA reports a bounded wait that ran out: `word` is the device-wide
+// error word the host reads back (kata_sync_status), written only with the
+// first code; `abort` is a flag in this CTA's shared memory that tells the
+// CTA's other roles to stop waiting. A stale device word from an earlier
+// launch therefore never stops a later one: only this CTA's own flag does.
+struct ErrCtx {
+    unsigned int *word;   // global memory
+    unsigned int *abort;  // shared memory, zeroed before the first wait
+};
+
+__device__ __forceinline__ bool cta_aborted(const ErrCtx &e) {
+    return *reinterpret_cast<volatile unsigned int *>(e.abort) != 0u;
+}
+
+__device__ __forceinline__ void report_timeout(const ErrCtx &e, unsigned int code) {
+    if (e.word) atomicCAS(e.word, 0u, code);
+    atomicExch(e.abort, code);
+}
+
+// Bounded wait: returns false (and records `code`) if the phase with this
+// parity has not completed after `limit` polls, or gives up early (without a
+// code of its own) once another role of the CTA has recorded one. A phase
+// that has already completed is seen by the cheap non-blocking probe; only a
+// wait that has to wait uses the suspending form.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const ErrCtx &err,
                                           unsigned int code, uint32_t limit = 1u << 22) {
     if (mbar_test_wait(bar, parity)) return true;
     for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (err && (i & 1023u) == 1023u && *((volatile unsigned int *)err) != 0u) return false;
+        if ((i & 1023u) == 1023u && cta_aborted(err)) return false;
     }
-    if (err) atomicCAS(err, 0u, code);
+    report_timeout(err, code);
     return false;
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  unsigned int *err, unsigned int code,
-                                                  uint32_t limit = 1u << 22) {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if (err && (i & 1023u) == 1023u && *((volatile unsigned int *)err) != 0u) return false;
-    }
-    if (err) atomicCAS(err, 0u, code);
+// Bounded wait for the teardown: waits for copies or MMAs this thread issued
+// itself, so it does not give up when another role aborts (only after its own
+// limit, recording `code`).
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, const ErrCtx &err,
+                                           unsigned int code, uint32_t limit = 1u << 22) {
+    if (mbar_test_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    report_timeout(err, code);
     return false;
+}
+
+// Named barrier `id` over `nthreads` threads that also ANDs a predicate over
+// them: every participant learns whether all of them are still fine.
+__device__ __forceinline__ bool bar_sync_and(int id, int nthreads, bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0u;
 }
 
 __device__ __forceinline__ void fence_barrier_init() {

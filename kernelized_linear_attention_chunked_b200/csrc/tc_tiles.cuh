@@ -39,7 +39,7 @@ struct Shape {
 };
 
 // One warp-uniform wait: lane 0 polls, the result is broadcast.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const ErrCtx &err,
                                           unsigned int code) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, err, code) ? 1 : 0;

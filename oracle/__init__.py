@@ -19,7 +19,6 @@ Sources, by page title and section:
 from __future__ import annotations
 
 import ctypes as C
-import os
 from pathlib import Path
 
 import numpy as np
@@ -42,6 +41,9 @@ def _load():
         from .build import build
         build()
     lib = C.CDLL(str(_LIB_PATH))
+    lib.oracle_threads.restype = C.c_int
+    lib.oracle_threads.argtypes = []
+    lib.oracle_set_threads.argtypes = [C.c_int]
     lib.oracle_packed_dim.restype = C.c_long
     lib.oracle_packed_dim.argtypes = [C.c_int]
     lib.oracle_packed_index.restype = C.c_long
@@ -83,12 +85,14 @@ def _ptr(a: np.ndarray):
     raise TypeError(a.dtype)
 
 
-def set_threads(n: int | None) -> None:
-    """Thread count for the OpenMP loops over heads (None: library default)."""
-    if n is None:
-        os.environ.pop("OMP_NUM_THREADS", None)
-    else:
-        os.environ["OMP_NUM_THREADS"] = str(n)
+def set_threads(n: int) -> None:
+    """Thread count for the OpenMP loops over heads."""
+    _load().oracle_set_threads(int(n))
+
+
+def threads() -> int:
+    """Threads the OpenMP loops over heads use now."""
+    return int(_load().oracle_threads())
 
 
 def packed_dim(d: int) -> int:

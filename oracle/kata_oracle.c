@@ -38,10 +38,15 @@
  *  R3 eps is added to the readout denominator and to the SRE denominator.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_API __attribute__((visibility("default")))
+
+/* Threads the *_heads loops below run on (OpenMP's setting; no arithmetic). */
+ORACLE_API int oracle_threads(void) { return omp_get_max_threads(); }
+ORACLE_API void oracle_set_threads(int n) { if (n > 0) omp_set_num_threads(n); }
 
 /* ---------------------------------------------------------------- phi ---- */
 

@@ -21,7 +21,7 @@ def header_functions():
 
 def test_header_symbols_exported_and_bound():
     names = header_functions()
-    assert len(names) == 23
+    assert len(names) == 24
     L = kata.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -164,3 +164,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_binding, "LIB_PATH", tmp_path / "missing.so")
     with pytest.raises(kata.KataError):
         _binding.lib()
+
+
+def test_forced_timeout_hook_validation():
+    L = kata.lib()
+    # quadratic form only (d = 32 or 64, T a multiple of 128); polls in [1, 2^20]
+    assert L.kata_test_forced_timeout(FAKE, FAKE, FAKE, 1, 1, 256, 16, 1e-6, FAKE, 64, None) == 2
+    assert L.kata_test_forced_timeout(FAKE, FAKE, FAKE, 1, 1, 192, 32, 1e-6, FAKE, 64, None) == 1
+    assert L.kata_test_forced_timeout(FAKE, FAKE, FAKE, 1, 1, 256, 32, 1e-6, FAKE, 0, None) == 1
+    assert L.kata_test_forced_timeout(FAKE, FAKE, FAKE, 1, 1, 256, 32, 1e-6, FAKE, 1 << 21,
+                                      None) == 1
+    assert L.kata_test_forced_timeout(FAKE, None, FAKE, 1, 1, 256, 32, 1e-6, FAKE, 64, None) == 1
+    assert kata.launch_count() == 0

@@ -152,7 +152,52 @@ def test_lola_schedule_small_d16_fp32():
     lola_parity(q, k, v, window=16, cache=24)
 
 
-def test_lola_config_first_segments():
+def test_lola_config_full_schedule():
+    # the LoLA workload at its own size: all 128 segments of all 16 heads, every
+    # one of the 127 kept sets (tie rule, lock-step adoption), every output row
+    # and the final state
     w = WORKLOADS["lola_b2_h8_t8192_d64"]
     q, k, v = recall_inputs(w.B, w.H, w.T, w.d, dtype=w.dtype, seed=w.seed)
-    lola_parity(q, k, v, window=w.window, cache=w.cache, segments=24)
+    o, res, adopted = lola_parity(q, k, v, window=w.window, cache=w.cache)
+    assert len(res["kept_pos"]) == w.T // w.window - 1
+    # fp32 arithmetic on the stored bf16 values: far inside the bf16 bar
+    assert rel_l2(o, res["o"]) < 1e-4
+    assert len(adopted) <= 2 * w.B * w.H  # divergences only at near-ties
+
+
+def hybrid_reference(q, k, v, seg0, nq, w0, ck, cv, nc, H0, s0, tau):
+    B, H, T, d = q.shape
+    cap = ck.shape[2]
+    want = np.zeros((B, H, T, d))
+    nh = B * H
+    qq, kk, vv = (x.double().numpy().reshape(nh, T, d) for x in (q, k, v))
+    cks = np.ascontiguousarray(ck.double().numpy().reshape(nh, cap, d))
+    cvs = np.ascontiguousarray(cv.double().numpy().reshape(nh, cap, d))
+    Hh = np.ascontiguousarray(H0.double().numpy().reshape(nh, -1, d))
+    sh = np.ascontiguousarray(s0.double().numpy().reshape(nh, -1))
+    oo = want.reshape(nh, T, d)
+    L = oracle._load()
+    p = oracle._ptr
+    L.oracle_hybrid_segment_heads(nh, p(qq), p(kk), p(vv), T, d, d, 1e-6, tau, w0, seg0, nq,
+                                  p(cks), p(cvs), nc, cap, p(Hh), p(sh), p(oo))
+    return want[:, :, seg0:seg0 + nq]
+
+
+@pytest.mark.parametrize("scale", [12.0, 40.0])
+def test_hybrid_readout_large_logits(scale):
+    # tau q.k up to scale^2 / 8 (18 and 200): past fp32's exp range (88) at the
+    # larger scale; the kernel's max shift keeps the quotient finite and exact
+    B, H, T, d = 1, 2, 256, 64
+    q, k, v = recall_inputs(B, H, T, d, dtype="f32", seed=15)
+    q, k = q * scale, k * scale
+    H0, s0 = oracle_state(B, H, d, 100, seed=16)
+    ck, cv, _ = candidate_inputs(B, H, 32, d, dtype="f32", seed=17)
+    seg0, nq, w0 = 128, 64, 64
+    o = kata.hybrid_readout(*cuda(q, k, v), seg0, nq, w0, *cuda(ck, cv), 32, *cuda(H0, s0),
+                            eps=1e-6)
+    kata.sync_status()
+    got = o[:, :, seg0:seg0 + nq]
+    assert torch.isfinite(got).all()
+    want = hybrid_reference(q, k, v, seg0, nq, w0, ck, cv, 32, H0, s0, d ** -0.5)
+    assert np.isfinite(want).all()
+    assert rel_l2(got, want) < REL_F32
