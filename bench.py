@@ -658,18 +658,25 @@ def bench_lola(kata, args, dev, stream, peaks, dist_on, world):
     ws = torch.empty(kata.lola_prefill_workspace_bytes(w.B, w.H, w.T, w.d, w.window, w.cache),
                      dtype=torch.uint8, device=dev)
 
-    def step(i):
+    def step(i, run="auto"):
         Hst.zero_()
         s.zero_()
         kata.lola_prefill(q, k, v, window=w.window, cache=w.cache, eps=w.eps, Hst=Hst, s=s,
-                          o=o, workspace=ws)
+                          o=o, workspace=ws, run=run)
 
-    step(0)
+    run = "fused" if kata.lola_fused_applies(torch.bfloat16, w.d, w.window, w.cache) \
+        else "segments"
+    for i in range(3):
+        step(i)
     barrier(dist_on)
     n0 = kata.launch_count()
-    n = 3
+    n = 10
     ms = max_over_ranks(time_events(step, n, stream), dist_on) / n
     launches = (kata.launch_count() - n0) // n
+    kata.sync_status()
+    # the same schedule as launches per segment, for comparison
+    step(0, "segments")
+    ms_seg = time_events(lambda i: step(i, "segments"), 2, stream) / 2
     kata.sync_status()
     # labelled state-streaming model: every update of every head reads and
     # writes that head's fp32 state once (2 x D (d+1) x 4 bytes)
@@ -680,7 +687,8 @@ def bench_lola(kata, args, dev, stream, peaks, dist_on, world):
                      "writes its 540,800-byte fp32 state once; the state fits in L2, so this "
                      "is a yardstick, not the bytes HBM moves")
     return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
-            "updates": updates, "gpu_launches_per_pass": launches, "roofline": roof,
+            "run": run, "updates": updates, "gpu_launches_per_pass": launches, "roofline": roof,
+            "segments_run_ms": ms_seg,
             "note": "includes two state zero-fills per pass (torch memset)"}
 
 

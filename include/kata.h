@@ -317,6 +317,40 @@ KATA_API int lola_prefill(const void *q, const void *k, const void *v, int dtype
                  int d, int window, int cache, float eps, float tau, float *o, float *Hst,
                  float *s, int *kept_pos, void *workspace, size_t ws_bytes, void *stream);
 
+/* How lola_prefill runs the schedule. */
+enum { LOLA_RUN_AUTO = 0, LOLA_RUN_SEGMENTS = 1, LOLA_RUN_FUSED = 2 };
+/* LOLA_RUN_FUSED with exactly n CTAs per (b, h), n = 5 .. 8 (tests, tuning). */
+#define LOLA_RUN_FUSED_NCL(n) (10 + (n))
+
+/*
+ * lola_prefill with the execution chosen by the caller; the results are the
+ * same up to fp32 rounding.
+ *   LOLA_RUN_SEGMENTS  a few launches per segment (readout, SRE scoring,
+ *                      top-k, merge, cache bookkeeping); any size above.
+ *   LOLA_RUN_FUSED     one launch for the whole sequence: a cluster of n CTAs
+ *                      per (b, h) keeps that head's fp32 state in shared memory
+ *                      (each CTA 1/n of the packed rows) from the first segment
+ *                      to the last, and writes it back once; n is the largest of
+ *                      8, 7, 6, 5 for which every head's cluster is resident at
+ *                      once on the device (8 if none is). A cached pair's
+ *                      phi(k)^T [H | s] is carried from update to update by the
+ *                      merged pairs, (k . k_m)^2 v_m [KATA s2.2], instead of
+ *                      being recomputed against the whole state. Sizes:
+ *                      window a multiple of 8 up to 64, 2*window + cache <= 256,
+ *                      d * element size <= 128 bytes (bf16 d <= 64, fp32 d <= 32);
+ *                      other sizes return KATA_ERR_UNSUPPORTED.
+ *   LOLA_RUN_AUTO      fused when the sizes allow it, segments otherwise
+ *                      (what lola_prefill does).
+ * lola_prefill_workspace_bytes() covers both.
+ */
+KATA_API int lola_prefill_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                             int T, int d, int window, int cache, float eps, float tau, float *o,
+                             float *Hst, float *s, int *kept_pos, void *workspace,
+                             size_t ws_bytes, void *stream, int run);
+
+/* 1 if LOLA_RUN_FUSED takes these sizes (LOLA_RUN_AUTO then runs it), else 0. */
+KATA_API int lola_prefill_fused_applies(int dtype, int d, int window, int cache);
+
 #ifdef __cplusplus
 }
 #endif

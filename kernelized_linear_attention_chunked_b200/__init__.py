@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     hybrid_readout,
     launch_count,
     lib,
+    lola_fused_applies,
     lola_prefill,
     lola_prefill_workspace_bytes,
     packed_dim,

@@ -53,7 +53,13 @@ SIGNATURES = {
     "lola_prefill_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "lola_prefill": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp, _vp,
                           _vp, _sz, _vp]),
+    "lola_prefill_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
+                             _vp, _vp, _sz, _vp, _i]),
+    "lola_prefill_fused_applies": (_i, [_i, _i, _i, _i]),
 }
+
+# lola_prefill_ex executions; "fusedN": the fused run with N CTAs per head
+LOLA_RUNS = {"auto": 0, "segments": 1, "fused": 2, **{f"fused{n}": 10 + n for n in (5, 6, 7, 8)}}
 
 _lib = None
 
@@ -257,9 +263,16 @@ def hybrid_readout(q, k, v, seg0: int, nq: int, w0: int, ck, cv, nc: int, Hst, s
     return o
 
 
+def lola_fused_applies(dtype, d: int, window: int, cache: int) -> bool:
+    """True when the one-launch (fused) schedule takes these sizes."""
+    return bool(lib().lola_prefill_fused_applies(_DTYPE[dtype], d, window, cache))
+
+
 def lola_prefill(q, k, v, window: int, cache: int, eps: float = 1e-6, tau: float | None = None,
-                 Hst=None, s=None, kept: bool = False, o=None, workspace=None, stream=None):
-    """The LoLA schedule over q, k, v [B, H, T, d]. Returns (o, H, s, kept_pos or None)."""
+                 Hst=None, s=None, kept: bool = False, o=None, workspace=None, stream=None,
+                 run: str = "auto"):
+    """The LoLA schedule over q, k, v [B, H, T, d]. Returns (o, H, s, kept_pos or None).
+    ``run``: "fused" (one launch), "segments" (launches per segment) or "auto"."""
     _dev(q, k, v, Hst, s)
     B, Hh, T, d = q.shape
     D = packed_dim(d)
@@ -276,9 +289,10 @@ def lola_prefill(q, k, v, window: int, cache: int, eps: float = 1e-6, tau: float
     L = lib()
     if workspace is None:
         workspace = _workspace(L.lola_prefill_workspace_bytes(B, Hh, T, d, window, cache), dev)
-    _check("lola_prefill", L.lola_prefill(
+    _check("lola_prefill_ex", L.lola_prefill_ex(
         _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hh, T, d, window, cache, eps, tau, _ptr(o),
-        _ptr(Hst), _ptr(s), _ptr(kp), _ptr(workspace), workspace.numel(), _stream(stream)))
+        _ptr(Hst), _ptr(s), _ptr(kp), _ptr(workspace), workspace.numel(), _stream(stream),
+        LOLA_RUNS[run]))
     return o, Hst, s, (None if kp is None else kp[..., :cache])
 
 

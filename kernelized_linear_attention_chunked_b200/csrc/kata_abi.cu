@@ -555,15 +555,37 @@ size_t lola_prefill_workspace_bytes(int B, int H, int T, int d, int window, int 
     if (check_common(KATA_F32, B, H, d) || window < 1 || window > 256 || cache < 0 ||
         window + cache > 1024)
         return 0;
-    return kata::lola_workspace_bytes(B, H, T, d, window, cache);
+    const size_t seg = kata::lola_workspace_bytes(B, H, T, d, window, cache);
+    const size_t fused = kata::lola_fused_scratch_bytes(B * H, d);
+    return seg > fused ? seg : fused;
+}
+
+int lola_prefill_fused_applies(int dtype, int d, int window, int cache) {
+    return kata::lola_fused_applies(dtype, d, window, cache) ? 1 : 0;
 }
 
 int lola_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int T,
                  int d, int window, int cache, float eps, float tau, float *o, float *Hst,
                  float *s, int *kept_pos, void *workspace, size_t ws_bytes, void *stream) {
+    return lola_prefill_ex(q, k, v, dtype, B, H, T, d, window, cache, eps, tau, o, Hst, s,
+                           kept_pos, workspace, ws_bytes, stream, LOLA_RUN_AUTO);
+}
+
+int lola_prefill_ex(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                    int T, int d, int window, int cache, float eps, float tau, float *o,
+                    float *Hst, float *s, int *kept_pos, void *workspace, size_t ws_bytes,
+                    void *stream, int run) {
     g_last_error[0] = 0;
     int st = check_common(dtype, B, H, d);
     if (st) return st;
+    int ncl = 0;  // CTAs per head of the fused run (0: chosen by occupancy)
+    if (run >= LOLA_RUN_FUSED_NCL(5) && run <= LOLA_RUN_FUSED_NCL(8)) {
+        ncl = run - LOLA_RUN_FUSED_NCL(0);
+        run = LOLA_RUN_FUSED;
+    }
+    if (run != LOLA_RUN_AUTO && run != LOLA_RUN_SEGMENTS && run != LOLA_RUN_FUSED)
+        return fail(KATA_ERR_INVALID_ARG,
+                    "run=%d: 0 (auto), 1 (segments), 2 (fused) or LOLA_RUN_FUSED_NCL(5..8)", run);
     if (window < 1 || window > 256 || cache < 0 || window + cache > 1024)
         return fail(KATA_ERR_INVALID_ARG, "window=%d cache=%d out of range", window, cache);
     if (T <= 0 || T % window)
@@ -576,13 +598,21 @@ int lola_prefill(const void *q, const void *k, const void *v, int dtype, int B, 
     KATA_REQUIRE_PTR(s);
     KATA_OPTIONAL_PTR(kept_pos);
     if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
-    const size_t need = kata::lola_workspace_bytes(B, H, T, d, window, cache);
+    const bool fused_ok = kata::lola_fused_applies(dtype, d, window, cache);
+    if (run == LOLA_RUN_FUSED && !fused_ok)
+        return fail(KATA_ERR_UNSUPPORTED, "fused LoLA schedule: window a multiple of 8 up to 64, "
+                                          "2*window + cache <= 256, d*elem_size <= 128");
+    const bool fused = run == LOLA_RUN_FUSED || (run == LOLA_RUN_AUTO && fused_ok);
+    const size_t need = fused ? kata::lola_fused_scratch_bytes(B * H, d)
+                              : kata::lola_workspace_bytes(B, H, T, d, window, cache);
     if (!workspace || ws_bytes < need)
         return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
     KATA_REQUIRE_PTR(workspace);
-    cudaError_t e = kata::lola_run(q, k, v, dtype, B, H, T, d, window, cache, eps, tau, o, Hst,
-                                   s, kept_pos, workspace, ws_bytes,
-                                   static_cast<cudaStream_t>(stream));
+    cudaError_t e =
+        fused ? kata::lola_fused(q, k, v, dtype, B * H, T, d, window, cache, eps, tau, o, Hst, s,
+                                 kept_pos, workspace, ncl, static_cast<cudaStream_t>(stream))
+              : kata::lola_run(q, k, v, dtype, B, H, T, d, window, cache, eps, tau, o, Hst, s,
+                               kept_pos, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "lola_prefill launch");
     return KATA_OK;
 }

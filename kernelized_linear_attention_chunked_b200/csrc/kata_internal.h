@@ -60,10 +60,21 @@ cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtyp
                            float eps, float tau, float *o, void *ws, size_t ws_bytes,
                            cudaStream_t stream);
 size_t lola_workspace_bytes(int B, int H, int T, int d, int window, int cache);
+// The schedule as segment-by-segment launches (any supported size).
 cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int B, int H,
                      int T, int d, int window, int cache, float eps, float tau, float *o,
                      float *Hst, float *s, int *kept_pos, void *ws, size_t ws_bytes,
                      cudaStream_t stream);
+
+// The schedule as one launch, a cluster of CTAs per head holding the state on
+// chip (lola_fused.cu): the sizes lola_fused_applies() accepts; the scratch is
+// lola_fused_scratch_bytes() of device memory. ncl = CTAs per head (5 to 8), or
+// 0: the largest that keeps every head's cluster resident at once.
+bool lola_fused_applies(int dtype, int d, int window, int cache);
+size_t lola_fused_scratch_bytes(int nh, int d);
+cudaError_t lola_fused(const void *q, const void *k, const void *v, int dtype, int nh, int T,
+                       int d, int window, int cache, float eps, float tau, float *o, float *Hst,
+                       float *s, int *kept_pos, void *scratch, int ncl, cudaStream_t stream);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
