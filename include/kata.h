@@ -319,7 +319,7 @@ KATA_API int lola_prefill(const void *q, const void *k, const void *v, int dtype
 
 /* How lola_prefill runs the schedule. */
 enum { LOLA_RUN_AUTO = 0, LOLA_RUN_SEGMENTS = 1, LOLA_RUN_FUSED = 2 };
-/* LOLA_RUN_FUSED with exactly n CTAs per (b, h), n = 5 .. 8 (tests, tuning). */
+/* LOLA_RUN_FUSED with exactly n CTAs per (b, h), n = 6 .. 8 (tests, tuning). */
 #define LOLA_RUN_FUSED_NCL(n) (10 + (n))
 
 /*
@@ -331,7 +331,7 @@ enum { LOLA_RUN_AUTO = 0, LOLA_RUN_SEGMENTS = 1, LOLA_RUN_FUSED = 2 };
  *                      per (b, h) keeps that head's fp32 state in shared memory
  *                      (each CTA 1/n of the packed rows) from the first segment
  *                      to the last, and writes it back once; n is the largest of
- *                      8, 7, 6, 5 for which every head's cluster is resident at
+ *                      8, 7, 6 for which every head's cluster is resident at
  *                      once on the device (8 if none is). A cached pair's
  *                      phi(k)^T [H | s] is carried from update to update by the
  *                      merged pairs, (k . k_m)^2 v_m [KATA s2.2], instead of

@@ -59,7 +59,7 @@ SIGNATURES = {
 }
 
 # lola_prefill_ex executions; "fusedN": the fused run with N CTAs per head
-LOLA_RUNS = {"auto": 0, "segments": 1, "fused": 2, **{f"fused{n}": 10 + n for n in (5, 6, 7, 8)}}
+LOLA_RUNS = {"auto": 0, "segments": 1, "fused": 2, **{f"fused{n}": 10 + n for n in (6, 7, 8)}}
 
 _lib = None
 

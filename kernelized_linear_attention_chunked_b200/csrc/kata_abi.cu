@@ -579,13 +579,13 @@ int lola_prefill_ex(const void *q, const void *k, const void *v, int dtype, int 
     int st = check_common(dtype, B, H, d);
     if (st) return st;
     int ncl = 0;  // CTAs per head of the fused run (0: chosen by occupancy)
-    if (run >= LOLA_RUN_FUSED_NCL(5) && run <= LOLA_RUN_FUSED_NCL(8)) {
+    if (run >= LOLA_RUN_FUSED_NCL(6) && run <= LOLA_RUN_FUSED_NCL(8)) {
         ncl = run - LOLA_RUN_FUSED_NCL(0);
         run = LOLA_RUN_FUSED;
     }
     if (run != LOLA_RUN_AUTO && run != LOLA_RUN_SEGMENTS && run != LOLA_RUN_FUSED)
         return fail(KATA_ERR_INVALID_ARG,
-                    "run=%d: 0 (auto), 1 (segments), 2 (fused) or LOLA_RUN_FUSED_NCL(5..8)", run);
+                    "run=%d: 0 (auto), 1 (segments), 2 (fused) or LOLA_RUN_FUSED_NCL(6..8)", run);
     if (window < 1 || window > 256 || cache < 0 || window + cache > 1024)
         return fail(KATA_ERR_INVALID_ARG, "window=%d cache=%d out of range", window, cache);
     if (T <= 0 || T % window)

@@ -68,7 +68,7 @@ cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int
 
 // The schedule as one launch, a cluster of CTAs per head holding the state on
 // chip (lola_fused.cu): the sizes lola_fused_applies() accepts; the scratch is
-// lola_fused_scratch_bytes() of device memory. ncl = CTAs per head (5 to 8), or
+// lola_fused_scratch_bytes() of device memory. ncl = CTAs per head (6 to 8), or
 // 0: the largest that keeps every head's cluster resident at once.
 bool lola_fused_applies(int dtype, int d, int window, int cache);
 size_t lola_fused_scratch_bytes(int nh, int d);

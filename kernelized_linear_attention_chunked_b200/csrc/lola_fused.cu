@@ -37,7 +37,7 @@
 //      cached candidate is never rescored against the whole state.
 // The state is written back once at the end.
 //
-// The cluster size NCL (8 down to 5) is the largest for which every head's
+// The cluster size NCL (8 down to 6) is the largest for which every head's
 // cluster is resident at once (a head whose cluster waits for a second wave
 // doubles the time of the whole launch).
 #include <atomic>
@@ -48,12 +48,14 @@
 namespace kata {
 namespace {
 
-constexpr int kFT = 288;          // threads: 8 warps for the H columns + 1 for s
+constexpr int kFT = 352;          // threads: a state row each in the merge (up to 352 rows);
+                                  // warps 0-7 score the H columns, warp 8 the s column
 constexpr int kRC = 32;           // state rows per phi chunk
 constexpr int kNSMax = 128;       // scoring vectors per segment (queries + new candidates)
 constexpr int kNKMax = 256;       // softmax keys per segment (window + cache)
 constexpr int kWMax = 64;         // longest segment
 constexpr int kQMax = 16;         // queries per CTA (a segment over at least 4 CTAs)
+constexpr int kNclMin = 6;        // fewest CTAs per head: D / 6 rows fit one pass of kFT threads
 constexpr int kVPT = 4;           // scoring vectors per thread (x 8 columns)
 
 __device__ __forceinline__ float xv(const float *p) { return *p; }
@@ -129,6 +131,7 @@ struct FusedCfg {
     static constexpr int NINT = 6 * kNKMax + 2 * kQMax;
     static constexpr size_t BYTES = (size_t)(OFF_INT + NINT) * 4;
     static_assert(OFF_SS % 4 == 0 && RED % 4 == 0 && BUF % 4 == 0, "16-byte alignment");
+    static_assert(R <= kFT, "one state row per thread in the merge");
 };
 
 // Global scratch per head: partial sums [NCL][kNSMax][DH+1], the full
@@ -483,8 +486,8 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             *reinterpret_cast<float4 *>(vm + mm * DH + a0 + 4) = make_float4(x[4], x[5], x[6], x[7]);
         }
         __syncthreads();
-        if (nm > 0 && tid < nrows) {
-            const int e = tab[tid];
+        for (int rr = tid; nm > 0 && rr < nrows; rr += kFT) {  // one pass: R <= kFT
+            const int e = tab[rr];
             const int a = e & 255, b = (e >> 8) & 255;
             const float wgt = (e >> 16) ? kSqrt2 : 1.f;
             float acc[DH];
@@ -506,7 +509,7 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 }
                 sacc += p;
             }
-            float4 *hr = reinterpret_cast<float4 *>(Hs + tid * DH);
+            float4 *hr = reinterpret_cast<float4 *>(Hs + rr * DH);
 #pragma unroll
             for (int c = 0; c < DH / 4; ++c) {
                 float4 h = hr[c];
@@ -516,7 +519,7 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 h.w += acc[4 * c + 3];
                 hr[c] = h;
             }
-            ss[tid] += sacc;
+            ss[rr] += sacc;
         }
         // kept candidate n (of this CTA's share): phi(k)^T [H | s] after the merge
         {
@@ -640,14 +643,14 @@ cudaError_t launch_ncl(const Tin *q, const Tin *k, const Tin *v, int nh, int T, 
     return after_launch();
 }
 
-// The largest cluster (8 down to 5 CTAs per head) that keeps every head's
+// The largest cluster (8 down to 6 CTAs per head) that keeps every head's
 // cluster resident at once; 8 when none does.
 template <typename Tin, int DH>
 int choose_ncl(int nh) {
+    static_assert(kNclMin == 6, "the candidates below");
     if (max_clusters<Tin, DH, 8>() >= nh) return 8;
     if (max_clusters<Tin, DH, 7>() >= nh) return 7;
     if (max_clusters<Tin, DH, 6>() >= nh) return 6;
-    if (max_clusters<Tin, DH, 5>() >= nh) return 5;
     return 8;
 }
 
@@ -660,7 +663,6 @@ cudaError_t launch_fused(const Tin *q, const Tin *k, const Tin *v, int nh, int T
         case 8: return launch_ncl<Tin, DH, 8>(q, k, v, nh, T, W, cache, eps, tau, o, Hst, s, kept_pos, scratch, stream);
         case 7: return launch_ncl<Tin, DH, 7>(q, k, v, nh, T, W, cache, eps, tau, o, Hst, s, kept_pos, scratch, stream);
         case 6: return launch_ncl<Tin, DH, 6>(q, k, v, nh, T, W, cache, eps, tau, o, Hst, s, kept_pos, scratch, stream);
-        case 5: return launch_ncl<Tin, DH, 5>(q, k, v, nh, T, W, cache, eps, tau, o, Hst, s, kept_pos, scratch, stream);
         default: return cudaErrorInvalidValue;
     }
 }
