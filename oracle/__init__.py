@@ -63,6 +63,16 @@ def _load():
                                                 C.c_int, C.c_double, C.c_double, C.c_long,
                                                 C.c_long, C.c_int, _dp, _dp, C.c_int, C.c_int,
                                                 _dp, _dp, _dp]
+    lib.oracle_feature_dim.restype = C.c_long
+    lib.oracle_feature_dim.argtypes = [C.c_int, C.c_int, C.c_int]
+    lib.oracle_phi_feature.argtypes = [_dp, C.c_int, C.c_int, C.c_int, _dp]
+    lib.oracle_kernel_feature.restype = C.c_double
+    lib.oracle_kernel_feature.argtypes = [_dp, _dp, C.c_int, C.c_int, C.c_int]
+    lib.oracle_quadratic_feature_heads.argtypes = [C.c_int, _dp, _dp, _dp, C.c_long, C.c_int,
+                                                   C.c_int, C.c_double, C.c_int, C.c_int, _dp]
+    lib.oracle_recurrent_feature_heads.argtypes = [C.c_int, _dp, _dp, _dp, C.c_long, C.c_int,
+                                                   C.c_int, C.c_double, C.c_int, C.c_int, _dp,
+                                                   _dp, _dp]
     _lib = lib
     return lib
 
@@ -155,6 +165,82 @@ def recurrent(q, k, v, eps: float, H0=None, s0=None, readout: bool = True):
                                    _ptr(s), _ptr(o))
     return (None if o is None else o.reshape(lead + (T, dv)),
             Hst.reshape(lead + (D, dv)), s.reshape(lead + (D,)))
+
+
+# Multi-factor features ("Kernelized Linear Attention ...", s2.3 "Variants",
+# reading R13 in kata_oracle.c): the head vector in g sub-vectors of d/g values;
+# Mg keeps the g rank-one PSD factors apart, Sigma-g sums them.
+FEATURES = {"m1": 0, "mg": 1, "sigmag": 2}
+
+
+def feature_dim(d: int, feature: str, g: int) -> int:
+    """Packed feature dimension of a variant (0: invalid)."""
+    return int(_load().oracle_feature_dim(d, FEATURES[feature], g))
+
+
+def phi_feature(x, feature: str, g: int) -> np.ndarray:
+    """Packed feature psi of every row of x [..., d] -> [..., feature_dim]."""
+    x = _f64(x)
+    d = x.shape[-1]
+    Df = feature_dim(d, feature, g)
+    assert Df > 0
+    rows = x.reshape(-1, d)
+    out = np.empty((rows.shape[0], Df))
+    lib = _load()
+    for i in range(rows.shape[0]):
+        r = np.ascontiguousarray(rows[i])
+        o = np.empty(Df)
+        lib.oracle_phi_feature(_ptr(r), d, FEATURES[feature], g, _ptr(o))
+        out[i] = o
+    return out.reshape(x.shape[:-1] + (Df,))
+
+
+def kernel_feature(q, k, feature: str, g: int) -> float:
+    """kappa(q, k) = <psi(q), psi(k)> from the sub-vectors' dot products."""
+    q, k = _f64(q).ravel(), _f64(k).ravel()
+    return float(_load().oracle_kernel_feature(_ptr(q), _ptr(k), q.shape[0], FEATURES[feature],
+                                               g))
+
+
+def quadratic_feature(q, k, v, eps: float, feature: str, g: int) -> np.ndarray:
+    """o_i = sum_{j<=i} kappa(q_i,k_j) v_j / (sum_{j<=i} kappa(q_i,k_j) + eps) for [..., T, d]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    lead = q.shape[:-2]
+    T, d = q.shape[-2:]
+    dv = v.shape[-1]
+    nh = int(np.prod(lead)) if lead else 1
+    assert feature_dim(d, feature, g) > 0
+    o = np.empty((nh, T, dv))
+    _load().oracle_quadratic_feature_heads(nh, _ptr(q), _ptr(k), _ptr(v), T, d, dv, eps,
+                                           FEATURES[feature], g, _ptr(o))
+    return o.reshape(lead + (T, dv))
+
+
+def recurrent_feature(q, k, v, eps: float, feature: str, g: int, H0=None, s0=None,
+                      readout: bool = True):
+    """Literal recurrent form with a variant's feature. Returns (o or None, H, s)."""
+    k, v = _f64(k), _f64(v)
+    lead = k.shape[:-2]
+    T, d = k.shape[-2:]
+    dv = v.shape[-1]
+    Df = feature_dim(d, feature, g)
+    assert Df > 0
+    nh = int(np.prod(lead)) if lead else 1
+    Hst = np.zeros((nh, Df, dv)) if H0 is None else _f64(H0).reshape(nh, Df, dv).copy()
+    s = np.zeros((nh, Df)) if s0 is None else _f64(s0).reshape(nh, Df).copy()
+    qq = _f64(q) if readout else None
+    o = np.empty((nh, T, dv)) if readout else None
+    _load().oracle_recurrent_feature_heads(nh, _ptr(qq), _ptr(k), _ptr(v), T, d, dv, eps,
+                                           FEATURES[feature], g, _ptr(Hst), _ptr(s), _ptr(o))
+    return (None if o is None else o.reshape(lead + (T, dv)),
+            Hst.reshape(lead + (Df, dv)), s.reshape(lead + (Df,)))
+
+
+def decode_feature(H0, s0, q, k, v, eps: float, feature: str, g: int):
+    """Decode steps with a variant's feature: q, k, v [steps, B, H, d]."""
+    q, k, v = (np.moveaxis(_f64(x), 0, -2) for x in (q, k, v))
+    o, Hst, s = recurrent_feature(q, k, v, eps, feature, g, H0=H0, s0=s0)
+    return np.moveaxis(o, -2, 0), Hst, s
 
 
 def decode(H0, s0, q, k, v, eps: float):

@@ -352,3 +352,162 @@ ORACLE_API void oracle_hybrid_segment_heads(int nh, const double *q, const doubl
         }
     }
 }
+
+/* ------------------------------------------- multi-factor features ----- */
+
+/*
+ * [KATA s2.3 "Variants": KATA-Mg (several PSD factors) and KATA-Sigma-g
+ * (summed PSD factors), which trade the state size against the packing.]
+ * The page names the variants but not how the factors are formed. Reading
+ * R13: the head vector u (d values) is cut into g contiguous sub-vectors
+ * u_r = u[r p .. r p + p - 1], p = d / g, and each gives the rank-one PSD
+ * factor u_r u_r^T of s2.2:
+ *   feature 0, M1:      psi(u) = u u^T                          kernel (q.k)^2
+ *   feature 1, Mg:      psi(u) = blockdiag(u_1 u_1^T, ..., u_g u_g^T)
+ *                       (the g factors kept apart)              kernel sum_r (q_r.k_r)^2
+ *   feature 2, Sigma-g: psi(u) = sum_r u_r u_r^T (the factors summed into
+ *                       one p x p PSD matrix)                   kernel sum_{r,s} (q_r.k_s)^2
+ * Both are PSD features, so every attention weight <psi(q), psi(k)>_F is
+ * non-negative; g = 1 gives M1 for both. Packing: each symmetric p x p block
+ * as the upper triangle with sqrt(2) on off-diagonal entries (R1); Mg's g
+ * blocks one after another (block r at rows r p(p+1)/2 ...).
+ */
+static int oracle_feature_ok(int d, int feature, int g)
+{
+    if (feature == 0) return g == 1;
+    return (feature == 1 || feature == 2) && g >= 1 && d % g == 0;
+}
+
+/* Feature dimension: d(d+1)/2 (M1), g p(p+1)/2 (Mg), p(p+1)/2 (Sigma-g); 0 if invalid. */
+ORACLE_API long oracle_feature_dim(int d, int feature, int g)
+{
+    if (!oracle_feature_ok(d, feature, g)) return 0;
+    if (feature == 0) return oracle_packed_dim(d);
+    int p = d / g;
+    return feature == 1 ? (long)g * oracle_packed_dim(p) : oracle_packed_dim(p);
+}
+
+/* psi(x) in the packed layout above (R13). */
+ORACLE_API void oracle_phi_feature(const double *x, int d, int feature, int g, double *phi)
+{
+    if (feature == 0) {
+        oracle_phi(x, d, phi);
+        return;
+    }
+    const int p = d / g;
+    const long Dp = oracle_packed_dim(p);
+    const double r2 = sqrt(2.0);
+    if (feature == 2)
+        for (long i = 0; i < Dp; ++i) phi[i] = 0.0;
+    for (int r = 0; r < g; ++r) {
+        const double *xr = x + (long)r * p;
+        double *dst = feature == 1 ? phi + (long)r * Dp : phi;
+        for (int a = 0; a < p; ++a)
+            for (int b = a; b < p; ++b) {
+                double w = (a == b) ? 1.0 : r2;
+                double val = w * xr[a] * xr[b];
+                long at = oracle_packed_index(p, a, b);
+                if (feature == 1) dst[at] = val; else dst[at] += val;
+            }
+    }
+}
+
+/* The kernel <psi(q), psi(k)> from the sub-vectors' dot products, no feature map (R13). */
+ORACLE_API double oracle_kernel_feature(const double *q, const double *k, int d, int feature,
+                                        int g)
+{
+    if (feature == 0) {
+        double dot = 0.0;
+        for (int a = 0; a < d; ++a) dot += q[a] * k[a];
+        return dot * dot;
+    }
+    const int p = d / g;
+    double sum = 0.0;
+    for (int r = 0; r < g; ++r)
+        for (int t = 0; t < g; ++t) {
+            if (feature == 1 && t != r) continue;  /* Mg: each factor with itself only */
+            double dot = 0.0;
+            for (int a = 0; a < p; ++a) dot += q[(long)r * p + a] * k[(long)t * p + a];
+            sum += dot * dot;
+        }
+    return sum;
+}
+
+/*
+ * Quadratic form with a variant's kernel (R2, R3, R13), one head:
+ *   o_i = sum_{j<=i} kappa(q_i, k_j) v_j / (sum_{j<=i} kappa(q_i, k_j) + eps).
+ */
+ORACLE_API void oracle_quadratic_feature(const double *q, const double *k, const double *v,
+                                         long T, int d, int dv, double eps, int feature, int g,
+                                         double *o)
+{
+    double *num = (double *)malloc(sizeof(double) * (size_t)dv);
+    for (long i = 0; i < T; ++i) {
+        double den = 0.0;
+        for (int e = 0; e < dv; ++e) num[e] = 0.0;
+        for (long j = 0; j <= i; ++j) {
+            double w = oracle_kernel_feature(q + i * d, k + j * d, d, feature, g);
+            den += w;
+            for (int e = 0; e < dv; ++e) num[e] += w * v[j * dv + e];
+        }
+        for (int e = 0; e < dv; ++e) o[i * dv + e] = num[e] / (den + eps);
+    }
+    free(num);
+}
+
+/*
+ * Literal recurrent form with a variant's feature (R2, R3, R13), one head:
+ *   H += psi(k_i) v_i^T; s += psi(k_i); o_i = psi(q_i)^T H / (psi(q_i)^T s + eps).
+ * Hst [Df, dv], s [Df] (Df = oracle_feature_dim) in and out; o may be NULL.
+ */
+ORACLE_API void oracle_recurrent_feature(const double *q, const double *k, const double *v,
+                                         long T, int d, int dv, double eps, int feature,
+                                         int g, double *Hst, double *s, double *o)
+{
+    long D = oracle_feature_dim(d, feature, g);
+    double *pk = (double *)malloc(sizeof(double) * (size_t)D);
+    double *pq = (double *)malloc(sizeof(double) * (size_t)D);
+    for (long i = 0; i < T; ++i) {
+        oracle_phi_feature(k + i * d, d, feature, g, pk);
+        for (long r = 0; r < D; ++r) {
+            for (int e = 0; e < dv; ++e) Hst[r * dv + e] += pk[r] * v[i * dv + e];
+            s[r] += pk[r];
+        }
+        if (!o) continue;
+        oracle_phi_feature(q + i * d, d, feature, g, pq);
+        double den = 0.0;
+        for (long r = 0; r < D; ++r) den += pq[r] * s[r];
+        for (int e = 0; e < dv; ++e) {
+            double num = 0.0;
+            for (long r = 0; r < D; ++r) num += pq[r] * Hst[r * dv + e];
+            o[i * dv + e] = num / (den + eps);
+        }
+    }
+    free(pk);
+    free(pq);
+}
+
+ORACLE_API void oracle_quadratic_feature_heads(int nh, const double *q, const double *k,
+                                               const double *v, long T, int d, int dv,
+                                               double eps, int feature, int g, double *o)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < nh; ++h)
+        oracle_quadratic_feature(q + (long)h * T * d, k + (long)h * T * d,
+                                 v + (long)h * T * dv, T, d, dv, eps, feature, g,
+                                 o + (long)h * T * dv);
+}
+
+ORACLE_API void oracle_recurrent_feature_heads(int nh, const double *q, const double *k,
+                                               const double *v, long T, int d, int dv,
+                                               double eps, int feature, int g, double *Hst,
+                                               double *s, double *o)
+{
+    long D = oracle_feature_dim(d, feature, g);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < nh; ++h)
+        oracle_recurrent_feature(q ? q + (long)h * T * d : NULL, k + (long)h * T * d,
+                                 v + (long)h * T * dv, T, d, dv, eps, feature, g,
+                                 Hst + (long)h * D * dv, s + (long)h * D,
+                                 o ? o + (long)h * T * dv : NULL);
+}

@@ -408,3 +408,143 @@ def test_lola_no_cache_state_is_evicted_prefix():
     num = w @ v[0, 0, 16:i + 1] + pq @ Hi[0, 0]
     den = w.sum() + pq @ si[0, 0] + 1e-6
     assert np.allclose(res["o"][0, 0, i], num / den, rtol=1e-12)
+
+
+# ---------------------------------------------- multi-factor features -----
+# KATA page s2.3 "Variants" (KATA-Mg: several PSD factors; KATA-Sigma-g: summed
+# PSD factors), reading R13: the head vector in g sub-vectors of p = d/g values.
+
+VARIANTS = [("mg", 2), ("mg", 4), ("sigmag", 2), ("sigmag", 4), ("mg", 1), ("sigmag", 1)]
+
+
+@pytest.mark.parametrize("feature,g", VARIANTS)
+def test_feature_dimension(feature, g):
+    d = 16
+    p = d // g
+    want = g * p * (p + 1) // 2 if feature == "mg" else p * (p + 1) // 2
+    assert oracle.feature_dim(d, feature, g) == want
+    assert oracle.feature_dim(16, "mg", 3) == 0  # g must divide d
+    assert oracle.feature_dim(16, "m1", 2) == 0
+
+
+def test_one_factor_is_the_rank_one_feature():
+    """g = 1: both variants are psi(u) = u u^T, i.e. M1 (pinned above)."""
+    x = np.random.default_rng(5).standard_normal((7, 16))
+    for feature in ("mg", "sigmag", "m1"):
+        assert np.array_equal(oracle.phi_feature(x, feature, 1), oracle.phi(x))
+
+
+@pytest.mark.parametrize("g", [2, 4, 8])
+def test_factor_features_built_from_the_rank_one_feature(g):
+    """Mg's feature is the pinned M1 feature of each sub-vector, in order;
+    Sigma-g's is their sum (independent of the oracle's own loops)."""
+    d = 16
+    p = d // g
+    x = np.random.default_rng(g).standard_normal((5, d))
+    parts = [oracle.phi(x[:, r * p:(r + 1) * p]) for r in range(g)]
+    assert np.allclose(oracle.phi_feature(x, "mg", g), np.concatenate(parts, axis=1),
+                       rtol=1e-15, atol=1e-15)
+    assert np.allclose(oracle.phi_feature(x, "sigmag", g), np.sum(parts, axis=0),
+                       rtol=1e-14, atol=1e-14)
+
+
+@pytest.mark.parametrize("feature,g", VARIANTS)
+def test_feature_inner_product_is_the_kernel(feature, g):
+    """<psi(x), psi(y)> (feature map) equals kappa(x, y) (sub-vector dot products)."""
+    rng = np.random.default_rng(17 + g)
+    for _ in range(20):
+        x, y = rng.standard_normal(16), rng.standard_normal(16)
+        lhs = float(oracle.phi_feature(x[None], feature, g)[0] @
+                    oracle.phi_feature(y[None], feature, g)[0])
+        rhs = oracle.kernel_feature(x, y, feature, g)
+        assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(rhs))
+        assert rhs >= 0.0  # PSD factors: non-negative weights
+
+
+def test_factor_kernels_distinguish_kept_apart_from_summed():
+    """A query living in factor 1 and a key living in factor 2: Mg has no
+    cross-factor term (weight 0), Sigma-g does ((q_1.k_2)^2); within one factor
+    both reduce to M1 on that sub-vector."""
+    d, g, p = 8, 2, 4
+    rng = np.random.default_rng(2)
+    a, b = rng.standard_normal(p), rng.standard_normal(p)
+    q = np.concatenate([a, np.zeros(p)])
+    k_other = np.concatenate([np.zeros(p), b])
+    k_same = np.concatenate([b, np.zeros(p)])
+    assert oracle.kernel_feature(q, k_other, "mg", g) == 0.0
+    assert np.isclose(oracle.kernel_feature(q, k_other, "sigmag", g), float(a @ b) ** 2,
+                      rtol=1e-14)
+    for feature in ("mg", "sigmag"):
+        assert np.isclose(oracle.kernel_feature(q, k_same, feature, g), float(a @ b) ** 2,
+                          rtol=1e-14)
+    # Mg of a full vector is the sum of M1 kernels of the sub-vectors
+    x, y = rng.standard_normal(d), rng.standard_normal(d)
+    m1 = sum(oracle.kernel_feature(x[r * p:(r + 1) * p], y[r * p:(r + 1) * p], "m1", 1)
+             for r in range(g))
+    assert np.isclose(oracle.kernel_feature(x, y, "mg", g), m1, rtol=1e-14)
+
+
+@pytest.mark.parametrize("feature,g", VARIANTS)
+def test_feature_quadratic_equals_recurrent(feature, g):
+    rng = np.random.default_rng(23 * g)
+    T, d, dv = 37, 16, 5
+    q, k, v = (rng.standard_normal((2, T, d)), rng.standard_normal((2, T, d)),
+               rng.standard_normal((2, T, dv)))
+    oq = oracle.quadratic_feature(q, k, v, 1e-6, feature, g)
+    orc, H, s = oracle.recurrent_feature(q, k, v, 1e-6, feature, g)
+    assert rel(orc, oq) < 1e-12
+    # the state is the sum of the key features (normaliser) and their v-outer products
+    pk = oracle.phi_feature(k, feature, g)
+    assert np.allclose(s, pk.sum(axis=1), rtol=1e-12, atol=1e-12)
+    assert np.allclose(H, np.einsum("htr,hte->hre", pk, v), rtol=1e-12, atol=1e-12)
+
+
+def _exact_factor_quadratic(q, k, v, eps, feature, g):
+    """Exact rationals: kappa from sub-vector dot products, inclusive causal sum."""
+    d = len(q[0])
+    p = d // g
+    out = []
+    for i in range(len(q)):
+        num = [Fraction(0)] * len(v[0])
+        den = Fraction(0)
+        for j in range(i + 1):
+            w = Fraction(0)
+            for r in range(g):
+                for t in range(g):
+                    if feature == "mg" and t != r:
+                        continue
+                    w += sum(Fraction(q[i][r * p + a]) * Fraction(k[j][t * p + a])
+                             for a in range(p)) ** 2
+            den += w
+            num = [n + w * Fraction(x) for n, x in zip(num, v[j])]
+        out.append([float(n / (den + eps)) for n in num])
+    return np.array(out)
+
+
+@pytest.mark.parametrize("feature,g", [("mg", 2), ("sigmag", 2), ("sigmag", 3)])
+def test_feature_exact_rational_brute_force(feature, g):
+    d = 6
+    rng = np.random.default_rng(41 + g)
+    T = 9
+    q = rng.integers(-3, 4, (T, d))
+    k = rng.integers(-3, 4, (T, d))
+    v = rng.integers(-5, 6, (T, 2))
+    eps = Fraction(1, 10 ** 6)
+    exact = _exact_factor_quadratic(q.tolist(), k.tolist(), v.tolist(), eps, feature, g)
+    for got in (oracle.quadratic_feature(q, k, v, 1e-6, feature, g),
+                oracle.recurrent_feature(q, k, v, 1e-6, feature, g)[0]):
+        assert np.allclose(got, exact, rtol=1e-12, atol=1e-12)
+
+
+def test_feature_decode_continues_recurrent():
+    rng = np.random.default_rng(9)
+    T0, T1, d = 20, 6, 16
+    q, k, v = (rng.standard_normal((3, T0 + T1, d)) for _ in range(3))
+    for feature, g in (("mg", 4), ("sigmag", 2)):
+        full, Hf, sf = oracle.recurrent_feature(q, k, v, 1e-6, feature, g)
+        _, H0, s0 = oracle.recurrent_feature(None, k[:, :T0], v[:, :T0], 1e-6, feature, g,
+                                             readout=False)
+        od, Hd, sd = oracle.decode_feature(H0, s0, *(np.moveaxis(x[:, T0:], 1, 0)
+                                                     for x in (q, k, v)), 1e-6, feature, g)
+        assert rel(np.moveaxis(od, 0, 1), full[:, T0:]) < 1e-12
+        assert rel(Hd, Hf) < 1e-12 and rel(sd, sf) < 1e-12
