@@ -194,6 +194,46 @@ KATA_API int kata_prefill_host(const void *q_host, const void *k_host, const voi
                       int B, int H, int T, int d, int chunk, float eps, float *o_host,
                       void *workspace, size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------ multi-factor features -- */
+
+/*
+ * The feature variants of [KATA s2.3 "Variants"]: KATA-Mg (several PSD
+ * factors) and KATA-Sigma-g (summed PSD factors). The page does not say how
+ * the factors are formed; this library reads them as follows. The head vector
+ * x (d values) is cut into g contiguous sub-vectors x_r of p = d/g values, and
+ * each gives the rank-one PSD factor x_r x_r^T of s2.2:
+ *   KATA_FEATURE_RANK1   psi(x) = x x^T (g = 1)          kernel (q.k)^2
+ *   KATA_FEATURE_MG      psi(x) = the g factors apart     kernel sum_r (q_r.k_r)^2
+ *   KATA_FEATURE_SIGMAG  psi(x) = sum_r x_r x_r^T         kernel sum_{r,t} (q_r.k_t)^2
+ * State layout: each symmetric p x p block as the packed upper triangle
+ * (sqrt(2) off the diagonal, as for the rank-one feature); Mg stores its g
+ * blocks one after another. The state has kata_feature_dim(d, feature, g)
+ * rows: d(d+1)/2, g p(p+1)/2 or p(p+1)/2. g must divide d with p >= 8.
+ */
+enum { KATA_FEATURE_RANK1 = 0, KATA_FEATURE_MG = 1, KATA_FEATURE_SIGMAG = 2 };
+
+/* Rows of the state of a feature (0: invalid d, feature or g). */
+KATA_API long kata_feature_dim(int d, int feature, int g);
+
+/*
+ * kata_prefill with a multi-factor feature: o_i = psi(q_i)^T H_i /
+ * (psi(q_i)^T s_i + eps), H_i = H_in + sum_{j<=i} psi(k_j) v_j^T, computed in
+ * the chunked form (intra-chunk kernel sum plus the carried state) on the CUDA
+ * cores in fp32, for fp32 or bf16 inputs. Arguments as kata_prefill, with
+ * H_in/H_out [B, H, Df, d] and s_in/s_out [B, H, Df], Df = kata_feature_dim().
+ * workspace: needed only when s_out aliases s_in (B*H*Df floats).
+ * KATA_FEATURE_RANK1 is kata_prefill itself.
+ */
+KATA_API int kata_prefill_feature(const void *q, const void *k, const void *v, int dtype, int B,
+                                  int H, int T, int d, int chunk, float eps, int feature, int g,
+                                  const float *H_in, const float *s_in, float *o, float *H_out,
+                                  float *s_out, void *workspace, size_t ws_bytes, void *stream);
+
+/* kata_decode_step with a multi-factor feature (state [B, H, Df, d], [B, H, Df]). */
+KATA_API int kata_decode_step_feature(const void *q, const void *k, const void *v, int dtype,
+                                      int B, int H, int d, float eps, int feature, int g,
+                                      float *Hst, float *s, float *o, void *stream);
+
 /* ---------------------------------------------------------------- decode -- */
 
 /*

@@ -12,6 +12,8 @@ from ._binding import (  # noqa: F401
     SIGNATURES,
     KataError,
     decode_step,
+    decode_step_feature,
+    feature_dim,
     decode_step_host,
     hybrid_readout,
     launch_count,
@@ -22,6 +24,7 @@ from ._binding import (  # noqa: F401
     packed_dim,
     prefill,
     prefill_auto_form,
+    prefill_feature,
     prefill_host,
     prefill_host_workspace_bytes,
     prefill_uses_tensor_cores,

@@ -56,7 +56,15 @@ SIGNATURES = {
     "lola_prefill_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _vp, _vp, _vp,
                              _vp, _vp, _sz, _vp, _i]),
     "lola_prefill_fused_applies": (_i, [_i, _i, _i, _i]),
+    "kata_feature_dim": (C.c_long, [_i, _i, _i]),
+    "kata_prefill_feature": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _vp,
+                                  _vp, _vp, _vp, _vp, _sz, _vp]),
+    "kata_decode_step_feature": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp, _vp, _vp,
+                                      _vp]),
 }
+
+# multi-factor features (kata_prefill_feature, kata_decode_step_feature)
+FEATURES = {"rank1": 0, "mg": 1, "sigmag": 2}
 
 # lola_prefill_ex executions; "fusedN": the fused run with N CTAs per head
 LOLA_RUNS = {"auto": 0, "segments": 1, "fused": 2, **{f"fused{n}": 10 + n for n in (6, 7, 8)}}
@@ -217,6 +225,48 @@ def decode_step(q, k, v, Hst, s, eps: float = 1e-6, o=None, stream=None):
     _check("kata_decode_step", lib().kata_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hh, d, eps, _ptr(Hst), _ptr(s), _ptr(o),
         _stream(stream)))
+    return o
+
+
+def feature_dim(d: int, feature: str, g: int) -> int:
+    """Rows of the state of a multi-factor feature (0: invalid)."""
+    return int(lib().kata_feature_dim(d, FEATURES[feature], g))
+
+
+def prefill_feature(q, k, v, feature: str, g: int, chunk: int = 64, eps: float = 1e-6,
+                    H_in=None, s_in=None, output: bool = True, state: bool = True,
+                    workspace=None, stream=None):
+    """Causal prefill with a multi-factor feature ("rank1", "mg", "sigmag").
+    Returns (o or None, H [B, H, Df, d] or None, s [B, H, Df] or None)."""
+    _dev(q, k, v, H_in, s_in)
+    B, Hh, T, d = q.shape
+    Df = feature_dim(d, feature, g)
+    if Df <= 0:
+        raise KataError(f"feature {feature!r} with g={g} is not available for d={d}")
+    o = torch.empty(B, Hh, T, d, dtype=torch.float32, device=q.device) if output else None
+    H_out = torch.empty(B, Hh, Df, d, dtype=torch.float32, device=q.device) if state else None
+    s_out = torch.empty(B, Hh, Df, dtype=torch.float32, device=q.device) if state else None
+    L = lib()
+    if workspace is None:
+        workspace = _workspace(L.kata_prefill_workspace_bytes(B, Hh, T, d, chunk, _dt(q)),
+                               q.device)
+    _check("kata_prefill_feature", L.kata_prefill_feature(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hh, T, d, chunk, eps, FEATURES[feature], g,
+        _ptr(H_in), _ptr(s_in), _ptr(o), _ptr(H_out), _ptr(s_out), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return o, H_out, s_out
+
+
+def decode_step_feature(q, k, v, Hst, s, feature: str, g: int, eps: float = 1e-6, o=None,
+                        stream=None):
+    """One decode step with a multi-factor feature, state updated in place. Returns o."""
+    _dev(q, k, v, Hst, s)
+    B, Hh, d = q.shape
+    if o is None:
+        o = torch.empty(B, Hh, d, dtype=torch.float32, device=q.device)
+    _check("kata_decode_step_feature", lib().kata_decode_step_feature(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hh, d, eps, FEATURES[feature], g, _ptr(Hst),
+        _ptr(s), _ptr(o), _stream(stream)))
     return o
 
 

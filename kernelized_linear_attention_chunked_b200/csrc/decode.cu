@@ -18,6 +18,10 @@
 // denominator into the first one's shared memory (distributed shared memory)
 // and the first writes o. phi(q) and phi(k) are built by all threads of each
 // CTA in shared memory.
+//
+// The multi-factor features of s2.3 "Variants" (KATA-Mg, KATA-Sigma-g;
+// kata_common.cuh) run through the same kernel with their own feature rows
+// (the state has D_f = feature_dim rows instead of D).
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
@@ -58,16 +62,17 @@ __device__ __forceinline__ void st_cluster(float *local, uint32_t cta, float v) 
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
-template <typename Tin, int DH>
+template <typename Tin, int DH, int FK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               float eps, float *__restrict__ Hst, float *__restrict__ s,
-              float *__restrict__ o) {
-    constexpr int D = DH * (DH + 1) / 2;
+              float *__restrict__ o, int g) {
+    constexpr int DM = DH * (DH + 1) / 2;  // the largest feature dimension (one factor)
+    const int D = FK == kFeatRank1 ? DM : feature_dim(DH, FK, g);
     constexpr int CG = DH / 4;           // float4 groups per row
     constexpr int RPP = kThreads / CG;   // rows per pass
     constexpr int NW = kThreads / 32;
-    __shared__ float pq[D], pk[D];
+    __shared__ float pq[DM], pk[DM];
     __shared__ float xs[3][DH];
     __shared__ float4 red[NW][CG];
     __shared__ float zred[NW];
@@ -81,13 +86,20 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
         xs[2][tid] = to_f32(v[(size_t)bh * DH + tid]);
     }
     __syncthreads();
-    for (int idx = tid; idx < DH * DH; idx += kThreads) {  // entry (a, b) of x x^T, b >= a
-        const int a = idx / DH, b = idx % DH;
-        if (b < a) continue;
-        const int at = packed_row_base(a, DH) + b - a;
-        const float w = (a == b) ? 1.f : kSqrt2;
-        pq[at] = (xs[0][a] * xs[0][b]) * w;
-        pk[at] = (xs[1][a] * xs[1][b]) * w;
+    if (FK == kFeatRank1) {
+        for (int idx = tid; idx < DH * DH; idx += kThreads) {  // entry (a, b) of x x^T, b >= a
+            const int a = idx / DH, b = idx % DH;
+            if (b < a) continue;
+            const int at = packed_row_base(a, DH) + b - a;
+            const float w = (a == b) ? 1.f : kSqrt2;
+            pq[at] = (xs[0][a] * xs[0][b]) * w;
+            pk[at] = (xs[1][a] * xs[1][b]) * w;
+        }
+    } else {
+        for (int r = tid; r < D; r += kThreads) {
+            pq[r] = factor_feature<FK>(xs[0], r, g, DH / g);
+            pk[r] = factor_feature<FK>(xs[1], r, g, DH / g);
+        }
     }
     __syncthreads();
     // announce that this CTA runs; the partner waits for it before writing into
@@ -160,27 +172,42 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     if (cr == 0 && tid < DH) o[(size_t)bh * DH + tid] = (num + xnum[tid]) / (zt + xz + eps);
 }
 
-template <typename Tin>
+template <typename Tin, int FK>
 cudaError_t launch(const void *q, const void *k, const void *v, int B, int H, int d, float eps,
-                   float *Hst, float *s, float *o, cudaStream_t stream) {
+                   float *Hst, float *s, float *o, int g, cudaStream_t stream) {
     dim3 grid(2 * B * H);  // clusters of two CTAs per head
     const Tin *qq = static_cast<const Tin *>(q), *kk = static_cast<const Tin *>(k),
               *vv = static_cast<const Tin *>(v);
     switch (d) {
-        case 16: decode_kernel<Tin, 16><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o); break;
-        case 32: decode_kernel<Tin, 32><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o); break;
-        case 64: decode_kernel<Tin, 64><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o); break;
+        case 16: decode_kernel<Tin, 16, FK><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o, g); break;
+        case 32: decode_kernel<Tin, 32, FK><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o, g); break;
+        case 64: decode_kernel<Tin, 64, FK><<<grid, kThreads, 0, stream>>>(qq, kk, vv, eps, Hst, s, o, g); break;
         default: return cudaErrorInvalidValue;
     }
     return after_launch();
 }
 
+template <typename Tin>
+cudaError_t launch_feature(const void *q, const void *k, const void *v, int B, int H, int d,
+                           float eps, float *Hst, float *s, float *o, int feature, int g,
+                           cudaStream_t stream) {
+    switch (feature) {
+        case kFeatRank1: return launch<Tin, kFeatRank1>(q, k, v, B, H, d, eps, Hst, s, o, 1, stream);
+        case kFeatMg: return launch<Tin, kFeatMg>(q, k, v, B, H, d, eps, Hst, s, o, g, stream);
+        case kFeatSigmaG: return launch<Tin, kFeatSigmaG>(q, k, v, B, H, d, eps, Hst, s, o, g, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
-                        int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream) {
-    return dtype == 0 ? launch<float>(q, k, v, B, H, d, eps, Hst, s, o, stream)
-                      : launch<__nv_bfloat16>(q, k, v, B, H, d, eps, Hst, s, o, stream);
+                        int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream,
+                        int feature, int g) {
+    return dtype == 0
+               ? launch_feature<float>(q, k, v, B, H, d, eps, Hst, s, o, feature, g, stream)
+               : launch_feature<__nv_bfloat16>(q, k, v, B, H, d, eps, Hst, s, o, feature, g,
+                                               stream);
 }
 
 }  // namespace kata

@@ -323,6 +323,70 @@ int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype) {
     return dtype == KATA_BF16 && kata::prefill_tc_supported(a) ? 1 : 0;
 }
 
+static int check_feature(int d, int feature, int g) {
+    if (feature == KATA_FEATURE_RANK1) {
+        if (g != 1) return fail(KATA_ERR_INVALID_ARG, "g=%d: the rank-one feature has g = 1", g);
+        return KATA_OK;
+    }
+    if (feature != KATA_FEATURE_MG && feature != KATA_FEATURE_SIGMAG)
+        return fail(KATA_ERR_UNSUPPORTED, "feature=%d: 0 (rank one), 1 (Mg) or 2 (Sigma-g)",
+                    feature);
+    if (g < 1 || d % g || d / g < 8)
+        return fail(KATA_ERR_UNSUPPORTED, "g=%d: must divide d=%d into factors of >= 8 values",
+                    g, d);
+    return KATA_OK;
+}
+
+long kata_feature_dim(int d, int feature, int g) {
+    if (d != 16 && d != 32 && d != 64) return 0;
+    if (check_feature(d, feature, g)) return 0;
+    return kata::feature_dim(d, feature, g);
+}
+
+int kata_prefill_feature(const void *q, const void *k, const void *v, int dtype, int B, int H,
+                         int T, int d, int chunk, float eps, int feature, int g,
+                         const float *H_in, const float *s_in, float *o, float *H_out,
+                         float *s_out, void *workspace, size_t ws_bytes, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_prefill(dtype, B, H, T, d, chunk);
+    if (st) return st;
+    if ((st = check_feature(d, feature, g))) return st;
+    if (feature == KATA_FEATURE_RANK1)
+        return kata_prefill_ex(q, k, v, dtype, B, H, T, d, chunk, eps, H_in, s_in, o, H_out,
+                               s_out, workspace, ws_bytes, stream, KATA_FORM_AUTO);
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_OPTIONAL_PTR(o);
+    KATA_OPTIONAL_PTR(H_in);
+    KATA_OPTIONAL_PTR(s_in);
+    KATA_OPTIONAL_PTR(H_out);
+    KATA_OPTIONAL_PTR(s_out);
+    if (!H_in != !s_in) return fail(KATA_ERR_INVALID_ARG, "H_in and s_in: both or neither");
+    if (!H_out != !s_out) return fail(KATA_ERR_INVALID_ARG, "H_out and s_out: both or neither");
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    const size_t s_bytes = (size_t)B * H * kata::feature_dim(d, feature, g) * sizeof(float);
+    const bool alias = s_in && s_out == s_in;
+    if (alias && (!workspace || ws_bytes < s_bytes))
+        return fail(KATA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, s_bytes);
+    KATA_OPTIONAL_PTR(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int *err = error_word();
+    if (!err) return fail(KATA_ERR_CUDA, "error word unavailable");
+    if (alias) {  // every CTA of a head reads s_in: keep a copy
+        cudaError_t e = cudaMemcpyAsync(workspace, s_in, s_bytes, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "copy s_in");
+        s_in = static_cast<const float *>(workspace);
+    }
+    kata::PrefillArgs a{q, k, v, dtype, B, H, T, d, chunk, eps, H_in, s_in, o, H_out, s_out,
+                        nullptr, 0, err};
+    a.feature = feature;
+    a.g = g;
+    cudaError_t e = kata::prefill_simt(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_prefill_feature launch");
+    return KATA_OK;
+}
+
 int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B, int H, int T,
                              int d, float eps, float *o, unsigned int polls, void *stream) {
     g_last_error[0] = 0;
@@ -401,6 +465,26 @@ int kata_decode_step(const void *q, const void *k, const void *v, int dtype, int
     cudaError_t e = kata::decode_step(q, k, v, dtype, B, H, d, eps, Hst, s, o,
                                       static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kata_decode_step launch");
+    return KATA_OK;
+}
+
+int kata_decode_step_feature(const void *q, const void *k, const void *v, int dtype, int B,
+                             int H, int d, float eps, int feature, int g, float *Hst, float *s,
+                             float *o, void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(dtype, B, H, d);
+    if (st) return st;
+    if ((st = check_feature(d, feature, g))) return st;
+    KATA_REQUIRE_PTR(q);
+    KATA_REQUIRE_PTR(k);
+    KATA_REQUIRE_PTR(v);
+    KATA_REQUIRE_PTR(Hst);
+    KATA_REQUIRE_PTR(s);
+    KATA_REQUIRE_PTR(o);
+    if (!(eps >= 0.f)) return fail(KATA_ERR_INVALID_ARG, "eps must be >= 0");
+    cudaError_t e = kata::decode_step(q, k, v, dtype, B, H, d, eps, Hst, s, o,
+                                      static_cast<cudaStream_t>(stream), feature, g);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_decode_step_feature launch");
     return KATA_OK;
 }
 

@@ -38,6 +38,65 @@ __device__ __forceinline__ float phi_entry(const float *x, uint16_t ab) {
     return a == b ? p : p * kSqrt2;
 }
 
+// Multi-factor features ("Kernelized Linear Attention", s2.3 "Variants":
+// KATA-Mg, several PSD factors; KATA-Sigma-g, summed PSD factors). The head
+// vector x is cut into g sub-vectors x_r of p = d/g values, each giving the
+// rank-one factor x_r x_r^T; Mg keeps the factors apart (g packed p x p
+// triangles one after another, kernel sum_r (q_r.k_r)^2), Sigma-g sums them
+// into one p x p matrix (kernel sum_{r,t} (q_r.k_t)^2). kFeatRank1 is the
+// single factor of s2.2.
+enum : int { kFeatRank1 = 0, kFeatMg = 1, kFeatSigmaG = 2 };
+
+__host__ __device__ __forceinline__ int feature_dim(int d, int feature, int g) {
+    const int p = d / g;
+    return feature == kFeatRank1 ? packed_dim(d)
+                                 : (feature == kFeatMg ? g * packed_dim(p) : packed_dim(p));
+}
+
+// Pair (a, b), a <= b < p, of packed row r of a p x p triangle.
+__device__ __forceinline__ void unpack_pair(int r, int p, int &a, int &b) {
+    a = 0;
+    while (packed_row_base(a + 1, p) <= r) ++a;
+    b = a + r - packed_row_base(a, p);
+}
+
+// Feature row r of x for Mg / Sigma-g (p = d / g), with sqrt(2) off the diagonal.
+template <int FK>
+__device__ __forceinline__ float factor_feature(const float *x, int r, int g, int p) {
+    const int Dp = packed_dim(p);
+    int a, b;
+    if (FK == kFeatMg) {
+        const int f = r / Dp;
+        unpack_pair(r - f * Dp, p, a, b);
+        const float v = x[f * p + a] * x[f * p + b];
+        return a == b ? v : v * kSqrt2;
+    }
+    unpack_pair(r, p, a, b);
+    float v = 0.f;
+    for (int t = 0; t < g; ++t) v = fmaf(x[t * p + a], x[t * p + b], v);
+    return a == b ? v : v * kSqrt2;
+}
+
+// kappa(q, k) = <psi(q), psi(k)> from the sub-vectors' dot products.
+template <int FK>
+__device__ __forceinline__ float factor_kernel(const float *q, const float *k, int d, int g) {
+    if (FK == kFeatRank1) {
+        float dot = 0.f;
+        for (int a = 0; a < d; ++a) dot = fmaf(q[a], k[a], dot);
+        return dot * dot;
+    }
+    const int p = d / g;
+    float sum = 0.f;
+    for (int r = 0; r < g; ++r)
+        for (int t = 0; t < g; ++t) {
+            if (FK == kFeatMg && t != r) continue;
+            float dot = 0.f;
+            for (int a = 0; a < p; ++a) dot = fmaf(q[r * p + a], k[t * p + a], dot);
+            sum = fmaf(dot, dot, sum);
+        }
+    return sum;
+}
+
 // Device-side error codes written to the per-device error word.
 enum : unsigned int { kErrNone = 0, kErrTimeout = 1 };
 

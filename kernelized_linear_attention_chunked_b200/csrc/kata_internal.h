@@ -16,6 +16,8 @@ struct PrefillArgs {
     void *ws;
     size_t ws_bytes;
     unsigned int *err;  // per-device error word
+    int feature = 0;    // kFeatRank1, kFeatMg or kFeatSigmaG (kata_common.cuh)
+    int g = 1;          // factors of a multi-factor feature
 };
 
 // fp32 CUDA-core path: any supported d and chunk, fp32 or bf16 inputs.
@@ -35,8 +37,10 @@ cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream);
 bool quad_tc_shape_ok(int dtype, int B, int H, int T, int d);
 cudaError_t quad_tc(const PrefillArgs &a, cudaStream_t stream, unsigned int stall = 0);
 
+// One decode step; feature / g select a multi-factor feature (kFeatRank1: s2.2's).
 cudaError_t decode_step(const void *q, const void *k, const void *v, int dtype, int B, int H,
-                        int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream);
+                        int d, float eps, float *Hst, float *s, float *o, cudaStream_t stream,
+                        int feature = 0, int g = 1);
 
 // LoLA pieces (lola.cu).
 size_t sre_workspace_bytes(int B, int H, int d, int n_cand);

@@ -12,6 +12,10 @@
 // normaliser s (D fp32) stay in shared memory for the whole sequence, so the
 // carry across chunks never leaves the SM. Every CTA of a head keeps an
 // identical copy of s (same operations in the same order).
+//
+// The same kernel runs the multi-factor features of s2.3 "Variants" (KATA-Mg,
+// KATA-Sigma-g; kata_common.cuh): only the feature rows and the intra-chunk
+// kernel change.
 #include "kata_common.cuh"
 #include "kata_internal.h"
 
@@ -24,21 +28,21 @@ constexpr int kRT = 16;  // packed rows per phi tile
 constexpr int kRTP = kRT + 1;
 constexpr int kCS = 64;  // tokens per inner chunk
 
-size_t simt_smem_bytes(int d) {
-    const int D = packed_dim(d);
+size_t simt_smem_bytes(int d, int D) {
     const size_t floats = (size_t)D * kE + D + 2 * (size_t)kCS * (d + 1) + (size_t)kCS * kE +
                           2 * (size_t)kCS * kRTP;
     return floats * sizeof(float) + ((size_t)D * sizeof(uint16_t) + 15) / 16 * 16;
 }
 
-template <typename Tin>
+template <typename Tin, int FK>
 __global__ void __launch_bounds__(kThreads)
 prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, int T, int d, int cs, float eps,
                     const float *__restrict__ H_in, const float *__restrict__ s_in,
                     float *__restrict__ o, float *__restrict__ H_out,
-                    float *__restrict__ s_out) {
-    const int D = packed_dim(d);
+                    float *__restrict__ s_out, int g) {
+    const int D = feature_dim(d, FK, g);
+    const int fp = d / g;  // values per factor
     const int NE = d / kE;
     const int bh = blockIdx.x / NE;
     const int e0 = (blockIdx.x % NE) * kE;
@@ -55,7 +59,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
     float *PK = PQ + kCS * kRTP;                   // [kCS][kRTP]
     uint16_t *tab = reinterpret_cast<uint16_t *>(PK + kCS * kRTP);
 
-    build_pair_table(tab, d);
+    if (FK == kFeatRank1) build_pair_table(tab, d);
     const size_t hoff = (size_t)bh * D * d;
     for (int idx = tid; idx < D * kE; idx += kThreads) {
         const int r = idx / kE, e = idx % kE;
@@ -84,10 +88,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         if (row < cs) {  // intra-chunk masked (q.k)^2 contraction
             const float *qi = Qs + row * dp;
             for (int j = 0; j <= row; ++j) {
-                const float *kj = Ks + j * dp;
-                float dot = 0.f;
-                for (int a = 0; a < d; ++a) dot = fmaf(qi[a], kj[a], dot);
-                const float w = dot * dot;
+                const float w = factor_kernel<FK>(qi, Ks + j * dp, d, g);
                 z += w;
                 const float *vj = Vs + j * kE + eq;
                 acc0 = fmaf(w, vj[0], acc0);
@@ -101,8 +102,13 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 const int i = idx / kRT, rr = idx % kRT, r = r0 + rr;
                 float pq = 0.f, pk = 0.f;
                 if (r < D) {
-                    pq = phi_entry(Qs + i * dp, tab[r]);
-                    pk = phi_entry(Ks + i * dp, tab[r]);
+                    if (FK == kFeatRank1) {
+                        pq = phi_entry(Qs + i * dp, tab[r]);
+                        pk = phi_entry(Ks + i * dp, tab[r]);
+                    } else {
+                        pq = factor_feature<FK>(Qs + i * dp, r, g, fp);
+                        pk = factor_feature<FK>(Ks + i * dp, r, g, fp);
+                    }
                 }
                 PQ[i * kRTP + rr] = pq;
                 PK[i * kRTP + rr] = pk;
@@ -156,26 +162,37 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
         for (int r = tid; r < D; r += kThreads) s_out[(size_t)bh * D + r] = sv[r];
 }
 
-template <typename Tin>
+template <typename Tin, int FK>
 cudaError_t launch_simt(const PrefillArgs &a, cudaStream_t stream) {
-    const size_t smem = simt_smem_bytes(a.d);
-    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<Tin>,
+    const size_t smem = simt_smem_bytes(a.d, feature_dim(a.d, FK, a.g));
+    cudaError_t err = cudaFuncSetAttribute(prefill_simt_kernel<Tin, FK>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
     const int cs = a.chunk < kCS ? a.chunk : kCS;
     dim3 grid(a.B * a.H * (a.d / kE));
-    prefill_simt_kernel<Tin><<<grid, kThreads, smem, stream>>>(
+    prefill_simt_kernel<Tin, FK><<<grid, kThreads, smem, stream>>>(
         static_cast<const Tin *>(a.q), static_cast<const Tin *>(a.k),
         static_cast<const Tin *>(a.v), a.T, a.d, cs, a.eps, a.H_in, a.s_in, a.o, a.H_out,
-        a.s_out);
+        a.s_out, a.g);
     return after_launch();
+}
+
+template <typename Tin>
+cudaError_t launch_feature(const PrefillArgs &a, cudaStream_t stream) {
+    switch (a.feature) {
+        case kFeatRank1: return launch_simt<Tin, kFeatRank1>(a, stream);
+        case kFeatMg: return launch_simt<Tin, kFeatMg>(a, stream);
+        case kFeatSigmaG: return launch_simt<Tin, kFeatSigmaG>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
 cudaError_t prefill_simt(const PrefillArgs &a, cudaStream_t stream) {
-    return a.dtype == 0 ? launch_simt<float>(a, stream) : launch_simt<__nv_bfloat16>(a, stream);
+    return a.dtype == 0 ? launch_feature<float>(a, stream)
+                        : launch_feature<__nv_bfloat16>(a, stream);
 }
 
 }  // namespace kata

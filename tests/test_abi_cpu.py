@@ -21,7 +21,7 @@ def header_functions():
 
 def test_header_symbols_exported_and_bound():
     names = header_functions()
-    assert len(names) == 26
+    assert len(names) == 29
     L = kata.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -175,4 +175,25 @@ def test_forced_timeout_hook_validation():
     assert L.kata_test_forced_timeout(FAKE, FAKE, FAKE, 1, 1, 256, 32, 1e-6, FAKE, 1 << 21,
                                       None) == 1
     assert L.kata_test_forced_timeout(FAKE, None, FAKE, 1, 1, 256, 32, 1e-6, FAKE, 64, None) == 1
+    assert kata.launch_count() == 0
+
+
+def test_feature_dims_and_validation():
+    L = kata.lib()
+    assert L.kata_feature_dim(64, 0, 1) == 2080
+    assert L.kata_feature_dim(64, 1, 2) == 2 * 528
+    assert L.kata_feature_dim(64, 2, 2) == 528
+    assert L.kata_feature_dim(64, 1, 8) == 8 * 36
+    assert L.kata_feature_dim(32, 2, 4) == 36
+    assert L.kata_feature_dim(64, 0, 2) == 0   # the rank-one feature has g = 1
+    assert L.kata_feature_dim(64, 1, 16) == 0  # factors of 4 values: too small
+    assert L.kata_feature_dim(48, 1, 2) == 0   # d not built
+    assert L.kata_feature_dim(64, 3, 2) == 0
+    # bad feature / g are refused before any launch
+    args = (FAKE, FAKE, FAKE, 1, 1, 2, 128, 32, 64, 1e-6)
+    assert L.kata_prefill_feature(*args, 3, 2, None, None, FAKE, None, None, None, 0, None) == 2
+    assert L.kata_prefill_feature(*args, 1, 8, None, None, FAKE, None, None, None, 0, None) == 2
+    assert L.kata_prefill_feature(*args, 1, 2, FAKE, None, FAKE, None, None, None, 0, None) == 1
+    assert L.kata_decode_step_feature(FAKE, FAKE, FAKE, 1, 1, 1, 32, 1e-6, 2, 3, FAKE, FAKE,
+                                      FAKE, None) == 2
     assert kata.launch_count() == 0
