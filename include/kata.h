@@ -234,6 +234,23 @@ KATA_API int kata_decode_step_feature(const void *q, const void *k, const void *
                                       int B, int H, int d, float eps, int feature, int g,
                                       float *Hst, float *s, float *o, void *stream);
 
+/* ------------------------------------------------- split sequences ------ */
+
+/*
+ * Exclusive prefix sums of states over the parts of a sequence [KATA s2.3:
+ * the state propagates across blocks as a prefix sum]. For a prefill whose
+ * sequence is split into nparts consecutive parts (one per device, say):
+ *   H_prefix[z] = H_parts[0] + ... + H_parts[z-1],  H_prefix[0] = 0,
+ * and the same for s, summed in part order; part z then runs kata_prefill
+ * with H_in = H_prefix[z], s_in = s_prefix[z] and gets the outputs and state
+ * of the whole sequence up to its end. H_parts, H_prefix [nparts, B, H, Df, d]
+ * and s_parts, s_prefix [nparts, B, H, Df] fp32, Df =
+ * kata_feature_dim(d, feature, g); the prefixes must not overwrite the parts.
+ */
+KATA_API int kata_state_prefix(const float *H_parts, const float *s_parts, int nparts, int B,
+                               int H, int d, int feature, int g, float *H_prefix,
+                               float *s_prefix, void *stream);
+
 /* ---------------------------------------------------------------- decode -- */
 
 /*

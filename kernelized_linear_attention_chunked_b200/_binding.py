@@ -61,6 +61,7 @@ SIGNATURES = {
                                   _vp, _vp, _vp, _vp, _sz, _vp]),
     "kata_decode_step_feature": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp, _vp, _vp,
                                       _vp]),
+    "kata_state_prefix": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
 
 # multi-factor features (kata_prefill_feature, kata_decode_step_feature)
@@ -268,6 +269,19 @@ def decode_step_feature(q, k, v, Hst, s, feature: str, g: int, eps: float = 1e-6
         _ptr(q), _ptr(k), _ptr(v), _dt(q), B, Hh, d, eps, FEATURES[feature], g, _ptr(Hst),
         _ptr(s), _ptr(o), _stream(stream)))
     return o
+
+
+def state_prefix(H_parts, s_parts, feature: str = "rank1", g: int = 1, stream=None):
+    """Exclusive prefix sums over the parts' states: H_parts [n, B, H, Df, d],
+    s_parts [n, B, H, Df] -> (H_prefix, s_prefix) of the same shapes, part z's
+    prefix the sum of parts 0 .. z-1."""
+    _dev(H_parts, s_parts)
+    n, B, Hh, Df, d = H_parts.shape
+    Hp, sp = torch.empty_like(H_parts), torch.empty_like(s_parts)
+    _check("kata_state_prefix", lib().kata_state_prefix(
+        _ptr(H_parts), _ptr(s_parts), n, B, Hh, d, FEATURES[feature], g, _ptr(Hp), _ptr(sp),
+        _stream(stream)))
+    return Hp, sp
 
 
 def decode_step_host(q, k, v, Hst, s, eps, o, workspace, stream=None) -> None:

@@ -387,6 +387,30 @@ int kata_prefill_feature(const void *q, const void *k, const void *v, int dtype,
     return KATA_OK;
 }
 
+int kata_state_prefix(const float *H_parts, const float *s_parts, int nparts, int B, int H,
+                      int d, int feature, int g, float *H_prefix, float *s_prefix,
+                      void *stream) {
+    g_last_error[0] = 0;
+    int st = check_common(KATA_F32, B, H, d);
+    if (st) return st;
+    if ((st = check_feature(d, feature, g))) return st;
+    if (nparts < 1 || nparts > 65536)
+        return fail(KATA_ERR_INVALID_ARG, "nparts=%d must be in [1, 65536]", nparts);
+    KATA_REQUIRE_PTR(H_parts);
+    KATA_REQUIRE_PTR(s_parts);
+    KATA_REQUIRE_PTR(H_prefix);
+    KATA_REQUIRE_PTR(s_prefix);
+    if (H_prefix == H_parts || s_prefix == s_parts)
+        return fail(KATA_ERR_INVALID_ARG, "the prefixes must not overwrite the parts");
+    const size_t Df = (size_t)kata::feature_dim(d, feature, g);
+    const size_t nH = (size_t)B * H * Df * d, ns = (size_t)B * H * Df;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = kata::exclusive_prefix(H_parts, nparts, nH, H_prefix, s);
+    if (e == cudaSuccess) e = kata::exclusive_prefix(s_parts, nparts, ns, s_prefix, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kata_state_prefix launch");
+    return KATA_OK;
+}
+
 int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B, int H, int T,
                              int d, float eps, float *o, unsigned int polls, void *stream) {
     g_last_error[0] = 0;

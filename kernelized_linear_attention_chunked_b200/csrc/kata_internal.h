@@ -80,6 +80,11 @@ cudaError_t lola_fused(const void *q, const void *k, const void *v, int dtype, i
                        int d, int window, int cache, float eps, float tau, float *o, float *Hst,
                        float *s, int *kept_pos, void *scratch, int ncl, cudaStream_t stream);
 
+// out[z] = in[0] + ... + in[z - 1] over nparts parts of n floats (n % 4 == 0,
+// 16-byte aligned), summed in part order (state_ops.cu).
+cudaError_t exclusive_prefix(const float *in, int nparts, size_t n, float *out,
+                             cudaStream_t stream);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Called right after every kernel launch: counts it (kata_launch_count) and

@@ -101,6 +101,13 @@ struct StateParams {
     float *H_out, *s_out;
     uint8_t *snap;  // [heads][nint][NS][NSNAP][128 B], or null: no snapshots
     unsigned int *err;
+    // Scan mode (several segments that write snapshots; seg_len a multiple of
+    // cpi): segment z >= 1 starts from the sum of the earlier segments' states,
+    // carry_H + (z - 1) * heads * D * d and carry_s + (z - 1) * heads * D,
+    // numbers its snapshot intervals from its first chunk's, and only the last
+    // segment writes H_out, s_out (the final state, not a partial).
+    const float *carry_H = nullptr, *carry_s = nullptr;
+    int scan = 0;
 };
 
 enum StateBar {
@@ -191,10 +198,25 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
     const int nch = p.nch - c0 < p.seg_len ? p.nch - c0 : p.seg_len;
     const long row0 = ((long)head * p.nch + c0) * kTile;  // first token row of this CTA
     constexpr int D = DH * (DH + 1) / 2;
-    float *H_out = p.H_out ? p.H_out + (size_t)blockIdx.z * gridDim.y * D * DH : nullptr;
-    float *s_out = p.s_out ? p.s_out + (size_t)blockIdx.z * gridDim.y * D : nullptr;
-    // the initial state enters through the first segment only
-    const float *H_in = blockIdx.z == 0 ? p.H_in : nullptr;
+    const int z = (int)blockIdx.z;
+    float *H_out, *s_out;
+    const float *H_in, *s_in;
+    if (p.scan) {
+        // scan mode: the state before chunk c0 comes in as this segment's
+        // initial state; the last segment's final state is the call's
+        const bool last = z == (int)gridDim.z - 1;
+        H_out = last ? p.H_out : nullptr;
+        s_out = last ? p.s_out : nullptr;
+        H_in = z == 0 ? p.H_in : p.carry_H + (size_t)(z - 1) * gridDim.y * D * DH;
+        s_in = z == 0 ? p.s_in : p.carry_s + (size_t)(z - 1) * gridDim.y * D;
+    } else {
+        H_out = p.H_out ? p.H_out + (size_t)z * gridDim.y * D * DH : nullptr;
+        s_out = p.s_out ? p.s_out + (size_t)z * gridDim.y * D : nullptr;
+        // the initial state enters through the first segment only
+        H_in = z == 0 ? p.H_in : nullptr;
+        s_in = z == 0 ? p.s_in : nullptr;
+    }
+    const int g0 = c0 / p.cpi;  // this segment's first snapshot interval
     // the readout kernel may start its setup and intra-chunk work now; it waits
     // for this grid's completion before it reads a snapshot
     if (threadIdx.x == 0) launch_dependents();
@@ -306,7 +328,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             const size_t hb = ((size_t)head * (DH * (DH + 1) / 2) + ci);
 #pragma unroll
             for (int n = 0; n < DH; ++n) init[n] = have ? H_in[hb * DH + n] * w : 0.f;
-            init[DH] = have ? p.s_in[hb] * w : 0.f;
+            init[DH] = have ? s_in[hb] * w : 0.f;
             uint32_t r[16];
 #pragma unroll
             for (int j = 0; j < S::NACC / 16; ++j) {
@@ -348,7 +370,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             return true;
         };
         bool ok = true;  // warp-uniform: every wait of this warp so far succeeded
-        if (H_in) ok = write_snapshot(0, init, ok);
+        if (H_in) ok = write_snapshot(g0, init, ok);
         if (f == 0) bulk_wait_read();
         // the state: sum of the issuers' accumulators, columns 0..DH-1 and s
         auto read_acc = [&](float (&x)[DH + 1]) {
@@ -442,7 +464,7 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
                 tc_fence_before();
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&bar[kSbSnap]);
-                ok = write_snapshot(c / p.cpi, x, ok);
+                ok = write_snapshot(g0 + c / p.cpi, x, ok);
             }
         }
         // final state, converted to the canonical layout
@@ -885,67 +907,141 @@ cudaError_t launch_state_sum(const float *part, int nseg, size_t n, float *out,
     return after_launch();
 }
 
+// In place over the segments' partial states part[z] (z = 0 .. nseg - 1, n4
+// float4s each): part[z] = part[0] + ... + part[z] for z < nseg - 1, in
+// segment order, so part[z - 1] becomes the state before segment z. The last
+// partial is not needed (the carry pass recomputes that segment from its carry).
+__global__ void __launch_bounds__(256) state_scan_kernel(float4 *__restrict__ part, int nseg,
+                                                         long n4) {
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
+         i += (long)gridDim.x * blockDim.x) {
+        float4 acc = part[i];
+        for (int z = 1; z < nseg - 1; ++z) {
+            const float4 x = part[(size_t)z * n4 + i];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+            part[(size_t)z * n4 + i] = acc;
+        }
+    }
+}
+
+cudaError_t launch_state_scan(float *part, int nseg, size_t n, cudaStream_t stream) {
+    const long n4 = (long)(n / 4);
+    const int blocks = (int)((n4 + 255) / 256 < 4 * 148 ? (n4 + 255) / 256 : 4 * 148);
+    state_scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4 *>(part), nseg, n4);
+    return after_launch();
+}
+
+// Sequence segments and their length for a call that writes snapshots (the
+// scan mode): whole snapshot intervals per segment, at least two segments.
+int scan_segments(int d, long nheads, int nch, int cpi, int &seg_len) {
+    const int want = state_segments(d, nheads, nch);
+    const int nint = nch / cpi;
+    if (want < 2 || nint < 2) return 1;
+    const int ipseg = (nint + want - 1) / want;  // intervals per segment
+    seg_len = ipseg * cpi;
+    return (nch + seg_len - 1) / seg_len;
+}
+
+template <int DH>
+cudaError_t launch_state(const CUtensorMap &mk, const CUtensorMap &mv, const StateParams &sp,
+                         int nheads, int nseg, cudaStream_t stream) {
+    // two issuers halve the MMA issue chain of a chunk; with d = 32 the
+    // accumulators are narrow enough to keep two Phi(K)^T slots as well
+    constexpr int NA = DH == 64 ? 1 : 2;
+    using L = StateCfg<DH, 2, NA>;
+    cudaError_t e = set_smem_once<state_kernel<DH, 2, NA>>(L::BYTES);
+    if (e != cudaSuccess) return e;
+    state_kernel<DH, 2, NA><<<dim3(Shape<DH>::NT, nheads, nseg), L::THREADS, L::BYTES, stream>>>(
+        mk, mv, sp);
+    return after_launch();
+}
+
 template <int DH>
 cudaError_t launch(const PrefillArgs &a, cudaStream_t stream) {
-    using S = Shape<DH>;
     const int nheads = a.B * a.H, nch = a.T / kTile;
     const int cpi = chunks_per_interval(DH, nch), nint = nch / cpi;
     const long rows = (long)nheads * a.T;
     const bool want_o = a.o != nullptr;
+    const size_t D = (size_t)DH * (DH + 1) / 2;
+    const size_t snap_bytes = want_o ? align_up(snapshot_bytes<DH>(nheads, nch), 256) : 0;
     uint8_t *snap = want_o ? static_cast<uint8_t *>(a.ws) : nullptr;
-    if (want_o && a.ws_bytes < snapshot_bytes<DH>(nheads, nch)) return cudaErrorInvalidValue;
+    if (want_o && a.ws_bytes < snap_bytes) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     if (!make_qkv_maps(&mq, &mk, &mv, a.q, a.k, a.v, DH, rows)) return cudaErrorInvalidValue;
 
     StateParams sp{nch, cpi, nint, nch, a.H_in, a.s_in, a.H_out, a.s_out, snap, a.err};
-    // a final-state-only pass: no interval ends inside the chunk loop, and the
-    // sequence split into segments when the tiles alone leave SMs idle (their
-    // partial states summed afterwards), if the workspace holds the partials
-    int nseg = 1;
-    float *pH = nullptr, *ps = nullptr;
+    // The sequence splits into segments across CTAs when the (tile, head) CTAs
+    // alone leave SMs idle and the workspace holds the segments' partial
+    // states (after the snapshots, if any):
+    //  - final state only: every segment accumulates its chunks from zero (the
+    //    first from H_in) and the partials are summed;
+    //  - with snapshots (the scan of the KATA page's s2.3, two-level): a first
+    //    pass computes each segment's partial state, an exclusive prefix over
+    //    the segments gives each segment the state before it, and a second pass
+    //    starts every segment from that carry and writes its snapshots.
+    int nseg = 1, seg_len = nch;
     if (!want_o) {
         sp.cpi = nch;
         sp.nint = 1;
         const int want = state_segments(DH, nheads, nch);
-        if (want > 1 && a.H_out && a.ws &&
-            a.ws_bytes >= partial_state_bytes(DH, nheads, want)) {
-            nseg = want;
-            sp.seg_len = (nch + nseg - 1) / nseg;
-            nseg = (nch + sp.seg_len - 1) / sp.seg_len;  // no empty segment
-            const size_t D = (size_t)DH * (DH + 1) / 2;
-            pH = static_cast<float *>(a.ws);
-            ps = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) +
-                                           align_up((size_t)nseg * nheads * D * DH * 4, 256));
-            sp.H_out = pH;
-            sp.s_out = ps;
+        if (want > 1) {
+            seg_len = (nch + want - 1) / want;
+            nseg = (nch + seg_len - 1) / seg_len;  // no empty segment
+        }
+    } else {
+        nseg = scan_segments(DH, nheads, nch, cpi, seg_len);
+    }
+    float *pH = nullptr, *ps = nullptr;
+    if (nseg > 1) {
+        const bool room = a.ws && a.ws_bytes >= snap_bytes + partial_state_bytes(DH, nheads, nseg);
+        // with snapshots, segment 0 rereads H_in in the second pass while the
+        // last segment writes H_out: an H_out that aliases H_in keeps one pass
+        const bool alias = want_o && a.H_in && a.H_out == a.H_in;
+        if (!room || alias || (!want_o && !a.H_out)) {
+            nseg = 1;
+            seg_len = nch;
+        } else {
+            uint8_t *base = static_cast<uint8_t *>(a.ws) + snap_bytes;
+            pH = reinterpret_cast<float *>(base);
+            ps = reinterpret_cast<float *>(base + align_up((size_t)nseg * nheads * D * DH * 4, 256));
         }
     }
-    {
-        // two issuers halve the MMA issue chain of a chunk; with d = 32 the
-        // accumulators are narrow enough to keep two Phi(K)^T slots as well
-        constexpr int NA = DH == 64 ? 1 : 2;
-        using L = StateCfg<DH, 2, NA>;
-        cudaError_t e = set_smem_once<state_kernel<DH, 2, NA>>(L::BYTES);
-        if (e != cudaSuccess) return e;
-        state_kernel<DH, 2, NA><<<dim3(S::NT, nheads, nseg), L::THREADS, L::BYTES, stream>>>(
-            mk, mv, sp);
-        e = after_launch();
-        if (e != cudaSuccess) return e;
-    }
+    sp.seg_len = seg_len;
+    cudaError_t e;
     if (nseg > 1) {
-        const size_t D = (size_t)DH * (DH + 1) / 2;
-        cudaError_t e = launch_state_sum(pH, nseg, (size_t)nheads * D * DH, a.H_out, stream);
-        if (e != cudaSuccess) return e;
-        e = launch_state_sum(ps, nseg, (size_t)nheads * D, a.s_out, stream);
-        if (e != cudaSuccess) return e;
+        // pass 1: each segment's partial state (no snapshots)
+        StateParams p1 = sp;
+        p1.cpi = nch;
+        p1.nint = 1;
+        p1.snap = nullptr;
+        p1.H_out = pH;
+        p1.s_out = ps;
+        if ((e = launch_state<DH>(mk, mv, p1, nheads, nseg, stream)) != cudaSuccess) return e;
+        if (!want_o) {
+            if ((e = launch_state_sum(pH, nseg, (size_t)nheads * D * DH, a.H_out, stream)) !=
+                cudaSuccess)
+                return e;
+            return launch_state_sum(ps, nseg, (size_t)nheads * D, a.s_out, stream);
+        }
+        // the state before each segment, then pass 2 from those carries
+        if ((e = launch_state_scan(pH, nseg, (size_t)nheads * D * DH, stream)) != cudaSuccess ||
+            (e = launch_state_scan(ps, nseg, (size_t)nheads * D, stream)) != cudaSuccess)
+            return e;
+        sp.scan = 1;
+        sp.carry_H = pH;
+        sp.carry_s = ps;
     }
+    if ((e = launch_state<DH>(mk, mv, sp, nheads, nseg, stream)) != cudaSuccess) return e;
     if (!want_o) return cudaSuccess;
     ReadParams rp{nch, cpi, nint, a.H_in != nullptr ? 1 : 0, snap, a.o, a.eps, a.err};
     // two issuers where the accumulators leave room for them (d = 32)
     constexpr int NIR = DH == 64 ? 1 : 2;
     using R = ReadCfg<DH, NIR>;
     auto kern = readout_kernel<DH, NIR>;
-    cudaError_t e = set_smem_once<readout_kernel<DH, NIR>>(R::BYTES);
+    e = set_smem_once<readout_kernel<DH, NIR>>(R::BYTES);
     if (e != cudaSuccess) return e;
     // programmatic dependent launch: overlap this grid's setup and intra-chunk
     // work with the end of the state kernel
@@ -979,9 +1075,15 @@ size_t prefill_tc_workspace_bytes(int B, int H, int T, int d, int) {
     if (T % kTile || (d != 32 && d != 64)) return 0;
     const long nheads = (long)B * H;
     const int nch = T / kTile;
-    const size_t snaps = d == 32 ? snapshot_bytes<32>(nheads, nch) : snapshot_bytes<64>(nheads, nch);
+    // a final-state-only call: the segments' partial states; a call with o:
+    // the snapshots, then the partial states of the scan's segments
+    const size_t snaps = align_up(d == 32 ? snapshot_bytes<32>(nheads, nch)
+                                          : snapshot_bytes<64>(nheads, nch), 256);
     const size_t parts = partial_state_bytes(d, nheads, state_segments(d, nheads, nch));
-    return snaps > parts ? snaps : parts;
+    int seg_len = nch;
+    const int nscan = scan_segments(d, nheads, nch, chunks_per_interval(d, nch), seg_len);
+    const size_t with_o = snaps + (nscan > 1 ? partial_state_bytes(d, nheads, nscan) : 0);
+    return with_o > parts ? with_o : parts;
 }
 
 cudaError_t prefill_tc(const PrefillArgs &a, cudaStream_t stream) {

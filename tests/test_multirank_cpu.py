@@ -52,3 +52,21 @@ def test_reference_arm_is_rank0_only(capsys):
     args = argparse.Namespace(gpus=2, steps=1, warmup=3)
     bench.run_reference(args, rank=1)
     assert capsys.readouterr().out == ""
+
+
+def test_context_parallel_gather_and_ranges_on_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ranks.gather_rank_main, args=(r, 2, port, queue))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    results = sorted(queue.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, stacked, rng in results:
+        # rank order on every rank: part 0 from rank 0, part 1 from rank 1
+        assert stacked == [[[1.0] * 3] * 2, [[2.0] * 3] * 2]
+        assert rng == (512 * rank, 512 * (rank + 1))
