@@ -31,6 +31,7 @@ from ._binding import (  # noqa: F401
     prefill_workspace_bytes,
     quadratic_max_tokens,
     sre_score_topk,
+    state_prefix,
     sync_status,
     test_forced_timeout,
 )

@@ -105,10 +105,12 @@ def test_output_and_final_state(d, T):
     assert rel_l2(o, ro) < tol("bf16")
     assert rel_l2(H, rH) < tol("bf16")
     assert rel_l2(s, rs) < tol("bf16")
-    # the same state as the chunked form's state pass computes (bit for bit)
+    # the same state as the chunked form computes (its passes sum the same
+    # fp32 terms, in another order when the sequence is split into segments)
     _, H2, s2 = kata.prefill(*cuda(q, k, v), chunk=64, form="chunked")
     kata.sync_status()
-    assert torch.equal(H, H2) and torch.equal(s, s2)
+    assert rel_l2(H, H2.double().cpu().numpy()) < 1e-5
+    assert rel_l2(s, s2.double().cpu().numpy()) < 1e-5
 
 
 def test_final_state_is_joined_back_to_the_callers_stream():
