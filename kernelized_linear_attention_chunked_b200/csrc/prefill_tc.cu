@@ -164,11 +164,11 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tile = blockIdx.x, head = blockIdx.y;
-    const ErrCtx err{p.err, tmem_slot + 1};
+    const ErrCtx err{p.err};
     constexpr int kTmaWarp = 4 + NI;
 
     if (threadIdx.x == 0) {
-        tmem_slot[1] = 0u;  // the CTA's abort flag
+        cta_abort_clear();
         for (int i = 0; i < 2; ++i) mbar_init(&bar[kSbDrain + i], 1);
         for (int i = 0; i < L::KR; ++i) {
             mbar_init(&bar[kSbKFull + i], 1);
@@ -457,10 +457,13 @@ __global__ void __launch_bounds__(StateCfg<DH, NI, NA>::THREADS,
             // chunk c opens interval g: the state after chunk c - 1 is snapshot g
             // (A(c) is already published, so the issuers wait only for this read)
             if (c > 0 && c % p.cpi == 0) {
-                if (ok) ok = warp_wait(&bar[kSbDone + (c - 1) % NA], ((c - 1) / NA) & 1, err, 0x422);
+                // after a failed wait this one gives up at once (the CTA's abort
+                // flag is set), and reading the allocated tensor memory is
+                // harmless: both stay unconditional, which keeps x in registers
+                ok = warp_wait(&bar[kSbDone + (c - 1) % NA], ((c - 1) / NA) & 1, err, 0x422) && ok;
                 tc_fence_after();
                 float x[DH + 1];
-                if (ok) read_acc(x);
+                read_acc(x);
                 tc_fence_before();
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&bar[kSbSnap]);
@@ -570,7 +573,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::SLOT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m = blockIdx.x, head = blockIdx.y;  // query tile, (batch, head)
-    const ErrCtx err{p.err, tmem_slot + 1};
+    const ErrCtx err{p.err};
 
     const int g = m / p.cpi;               // snapshot interval of this query tile
     const int kt0 = g * p.cpi;             // first key tile of the interval
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(ReadCfg<DH, NIR>::THREADS, 2)
             const bool four = i == kRbSFree || (i >= kRbAqFull && i < kRbAqFull + kRQMax);
             mbar_init(&bar[i], four ? 4 : (i == kRbODone ? NIR : 1));
         }
-        tmem_slot[1] = 0u;  // the CTA's abort flag
+        cta_abort_clear();
         fence_barrier_init();
     }
     if (warp == 4) {

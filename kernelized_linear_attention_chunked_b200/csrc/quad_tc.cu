@@ -115,14 +115,14 @@ __global__ void __launch_bounds__(QuadCfg<DH>::THREADS, 2)
     const int m = p.nch - 1 - (int)blockIdx.y;  // query tile: the longest rows launch first
     const int nh = 2 * (m + 1);                 // 64-key halves up to the diagonal
     const long row0 = (long)head * p.nch * kTile;
-    const ErrCtx err{p.err, tmem_slot + 1};
+    const ErrCtx err{p.err};
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQbCount; ++i) {
             const bool four = (i >= kQbSFree && i < kQbSFree + 2) || (i >= kQbPFull && i < kQbPFull + 2);
             mbar_init(&bar[i], four ? 4 : 1);
         }
-        tmem_slot[1] = 0u;  // the CTA's abort flag
+        cta_abort_clear();
         fence_barrier_init();
     }
     if (warp == L::ISSUER_WARP) {

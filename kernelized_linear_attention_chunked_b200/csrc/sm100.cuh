@@ -70,21 +70,28 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 
 // Where a CTA reports a bounded wait that ran out: `word` is the device-wide
 // error word the host reads back (kata_sync_status), written only with the
-// first code; `abort` is a flag in this CTA's shared memory that tells the
-// CTA's other roles to stop waiting. A stale device word from an earlier
-// launch therefore never stops a later one: only this CTA's own flag does.
+// first code; the CTA's abort flag (a shared-memory variable, cta_abort())
+// tells the CTA's other roles to stop waiting. A stale device word from an
+// earlier launch therefore never stops a later one: only this CTA's own flag
+// does. The flag sits at a fixed shared address, so it costs no register.
 struct ErrCtx {
-    unsigned int *word;   // global memory
-    unsigned int *abort;  // shared memory, zeroed before the first wait
+    unsigned int *word;  // global memory
 };
 
-__device__ __forceinline__ bool cta_aborted(const ErrCtx &e) {
-    return *reinterpret_cast<volatile unsigned int *>(e.abort) != 0u;
+// This CTA's abort flag; cta_abort_clear() runs before the CTA's first wait.
+__device__ __forceinline__ unsigned int *cta_abort() {
+    __shared__ unsigned int flag;
+    return &flag;
+}
+__device__ __forceinline__ void cta_abort_clear() { *cta_abort() = 0u; }
+
+__device__ __forceinline__ bool cta_aborted(const ErrCtx &) {
+    return *reinterpret_cast<volatile unsigned int *>(cta_abort()) != 0u;
 }
 
 __device__ __forceinline__ void report_timeout(const ErrCtx &e, unsigned int code) {
     if (e.word) atomicCAS(e.word, 0u, code);
-    atomicExch(e.abort, code);
+    atomicExch(cta_abort(), code);
 }
 
 // Bounded wait: returns false (and records `code`) if the phase with this
