@@ -114,6 +114,8 @@ size_t elem_bytes(int dtype) { return dtype == KATA_F32 ? 4 : 2; }
 
 }  // namespace
 
+unsigned int *kata::device_error_word() { return error_word(); }
+
 cudaError_t kata::after_launch() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError();

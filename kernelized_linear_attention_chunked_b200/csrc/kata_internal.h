@@ -58,6 +58,16 @@ cudaError_t sre_score_topk_noalloc(const float *Hst, const float *s, const void 
                                    float *scores, int *keep_idx, float *Hst_mut, float *s_mut,
                                    cudaStream_t stream);
 size_t readout_workspace_bytes(int B, int H, int d, int nq);
+// The SRE step on the tensor cores (sre_tc.cu): bf16 candidates, d = 32 or
+// 64, 1 <= n <= 256, 16-byte aligned state buffers; no workspace.
+bool sre_tc_applies(int dtype, int d, int n, const float *Hst, const float *s,
+                    const float *Hst_mut, const float *s_mut);
+cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void *vc,
+                   const int *pos, int nh, int d, int n, int cand_stride, int keep, float eps,
+                   int merge, float *scores, int *keep_idx, float *Hst_mut, float *s_mut,
+                   unsigned int *err, cudaStream_t stream);
+// This device's error word (kata_abi.cu): kernels record a timed-out wait there.
+unsigned int *device_error_word();
 cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtype, int B,
                            int H, int T, int d, int seg0, int nq, int w0, const void *ck,
                            const void *cv, int nc, int cap, const float *Hst, const float *s,

@@ -675,9 +675,8 @@ cudaError_t lola_impl(const Tin *q, const Tin *k, const Tin *v, int dtype, int n
         if ((err = after_launch()) != cudaSuccess) return err;
         const int n = nc + U;
         const int m = cache < n ? cache : n;
-        err = sre_impl<Tin>(Hst, s, static_cast<const Tin *>(w.ck[cur]),
-                            static_cast<const Tin *>(w.cv[cur]), w.cpos[cur], nh, d, n, cap,
-                            cache, eps, 1, nullptr, w.keep_idx, Hst, s, w.sre_ws, stream);
+        err = sre_score_topk(Hst, s, w.ck[cur], w.cv[cur], w.cpos[cur], dtype, nh, 1, d, n, cap,
+                             cache, eps, 1, nullptr, w.keep_idx, Hst, s, w.sre_ws, 0, stream);
         if (err != cudaSuccess) return err;
         lola_compact_kernel<Tin><<<nh, 256, 0, stream>>>(
             static_cast<const Tin *>(w.ck[cur]), static_cast<const Tin *>(w.cv[cur]),
@@ -725,6 +724,9 @@ cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, con
                            size_t ws_bytes, cudaStream_t stream) {
     (void)ws_bytes;
     const int nh = B * H;
+    if (sre_tc_applies(dtype, d, n_cand, Hst, s, Hst_mut, s_mut))
+        return sre_tc(Hst, s, kc, vc, pos, nh, d, n_cand, cand_stride, keep, eps, merge, scores,
+                      keep_idx, Hst_mut, s_mut, device_error_word(), stream);
     if (dtype == 0)
         return sre_impl<float>(Hst, s, static_cast<const float *>(kc),
                                static_cast<const float *>(vc), pos, nh, d, n_cand, cand_stride,

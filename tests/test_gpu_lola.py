@@ -20,7 +20,8 @@ def oracle_state(B, H, d, tokens, seed):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("d,n,keep", [(16, 40, 25), (64, 192, 128), (32, 70, 200), (64, 130, 0)])
+@pytest.mark.parametrize("d,n,keep", [(16, 40, 25), (64, 192, 128), (32, 70, 200), (64, 130, 0),
+                                        (64, 5, 2), (32, 17, 3), (64, 256, 100)])
 def test_sre_topk_merge(dtype, d, n, keep):
     B, H = 2, 3
     H0, s0 = oracle_state(B, H, d, 300, seed=d)
@@ -42,11 +43,11 @@ def test_sre_topk_merge(dtype, d, n, keep):
     assert rel_l2(Hg, Hr) < 1e-5 and rel_l2(sg, sr) < 1e-5
 
 
-@pytest.mark.parametrize("d", [32, 64])
-def test_sre_topk_merge_many_heads(d):
-    # 320 heads: enough (head, slice) pairs that one CTA scores every candidate
-    # against its slice of the state (the state is read once)
-    B, H, n, keep = 8, 40, 130, 64
+@pytest.mark.parametrize("d,n,keep", [(32, 130, 64), (64, 130, 64), (64, 192, 128), (64, 256, 0)])
+def test_sre_topk_merge_many_heads(d, n, keep):
+    # 320 heads: more CTAs than SMs on either path (several per SM over the
+    # launch), and enough (head, slice) pairs for the partial-sum path
+    B, H = 8, 40
     H0, s0 = oracle_state(B, H, d, 100, seed=d + 1)
     kc, vc, pos = candidate_inputs(B, H, n, d, dtype="bf16", seed=n + d)
     Hg, sg = cuda(H0.clone(), s0.clone())
@@ -62,6 +63,22 @@ def test_sre_topk_merge_many_heads(d):
     Hr, sr = H0.double().numpy().copy(), s0.double().numpy().copy()
     oracle.merge(Hr, sr, kc, vc, ki)
     assert rel_l2(Hg, Hr) < 1e-5 and rel_l2(sg, sr) < 1e-5
+
+
+def test_sre_merge_out_of_place():
+    # the merged state goes to separate buffers; the input state is untouched
+    B, H, n, d, keep = 2, 5, 100, 64, 40
+    H0, s0 = oracle_state(B, H, d, 200, seed=9)
+    kc, vc, pos = candidate_inputs(B, H, n, d, dtype="bf16", seed=10)
+    Hg, sg = cuda(H0.clone(), s0.clone())
+    Ho, so = torch.full_like(Hg, float("nan")), torch.full_like(sg, float("nan"))
+    _, ki = kata.sre_score_topk(Hg, sg, *cuda(kc, vc, pos), keep=keep, merge=True,
+                                Hst_mut=Ho, s_mut=so)
+    kata.sync_status()
+    assert torch.equal(Hg.cpu(), H0) and torch.equal(sg.cpu(), s0)
+    Hr, sr = H0.double().numpy().copy(), s0.double().numpy().copy()
+    oracle.merge(Hr, sr, kc, vc, ki.cpu().numpy())
+    assert rel_l2(Ho, Hr) < 1e-5 and rel_l2(so, sr) < 1e-5
 
 
 def test_sre_ties_go_to_smaller_position():
