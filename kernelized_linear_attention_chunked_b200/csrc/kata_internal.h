@@ -59,9 +59,9 @@ cudaError_t sre_score_topk_noalloc(const float *Hst, const float *s, const void 
                                    cudaStream_t stream);
 size_t readout_workspace_bytes(int B, int H, int d, int nq);
 // The SRE step on the tensor cores (sre_tc.cu): bf16 candidates, d = 32 or
-// 64, 1 <= n <= 256, 16-byte aligned state buffers; no workspace.
+// 64, 1 <= n <= 256, 16-byte aligned state and candidate buffers; no workspace.
 bool sre_tc_applies(int dtype, int d, int n, const float *Hst, const float *s,
-                    const float *Hst_mut, const float *s_mut);
+                    const float *Hst_mut, const float *s_mut, const void *kc, const void *vc);
 cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void *vc,
                    const int *pos, int nh, int d, int n, int cand_stride, int keep, float eps,
                    int merge, float *scores, int *keep_idx, float *Hst_mut, float *s_mut,

@@ -724,7 +724,7 @@ cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, con
                            size_t ws_bytes, cudaStream_t stream) {
     (void)ws_bytes;
     const int nh = B * H;
-    if (sre_tc_applies(dtype, d, n_cand, Hst, s, Hst_mut, s_mut))
+    if (sre_tc_applies(dtype, d, n_cand, Hst, s, Hst_mut, s_mut, kc, vc))
         return sre_tc(Hst, s, kc, vc, pos, nh, d, n_cand, cand_stride, keep, eps, merge, scores,
                       keep_idx, Hst_mut, s_mut, device_error_word(), stream);
     if (dtype == 0)

@@ -1,5 +1,4 @@
-// SRE scoring, top-k retention and merge on the tcgen05 tensor cores, with
-// split bf16 operands so that the scores keep fp32-level accuracy.
+// SRE scoring, top-k retention and merge on the tcgen05 tensor cores.
 //
 // "LoLA: Low-Rank Linear Attention with Sparse Caching", "Self-Recall Error":
 //   SRE_j = || phi(k_j)^T H / (phi(k_j)^T s + eps) - v_j ||^2,
@@ -9,23 +8,26 @@
 // Cones", s2.2, in the packed layout: row r is the pair (a, b), a <= b, and
 // phi(x)_r = w_r x_a x_b with w_r = sqrt(2) off the diagonal.
 //
-// One CTA per head (bf16 candidates, d = 32 or 64, at most 256 of them):
-//  1. Scores. For 32 packed rows at a time, D[m][c] += A[m][r] B[c][r] with
-//     A = (w [H | s])^T (m < d: a value column; m = d: the normaliser) and
-//     B[c][r] = k_c[a_r] k_c[b_r]. The product of two bf16 values is exact in
-//     fp32 and splits exactly into two bf16 parts (hi + lo); w [H | s] splits
-//     into hi + lo with a relative residual below 2^-16. Three MMAs per step
-//     (hi.hi, hi.lo, lo.hi) accumulate in fp32 tensor memory; what is dropped
-//     is below 2^-16 of each term, and the SRE, a distance of order |v|^2, is
-//     insensitive to that (1e-7 relative on the synthetic candidates). The
-//     state streams from HBM once, in 64-row bulk copies, three in flight.
-//  2. The SRE of every candidate from D (numerator lanes, normaliser lane),
-//     then the kept set (higher SRE, then smaller position, then slot) in
-//     ascending position, and the list of candidates to merge.
-//  3. Merge, 128 packed rows at a time: D2[r][e] = sum_m k_m[a_r] k_m[b_r]
-//     [v_m | 1][e] with exact products (two bf16 parts times bf16 values and
-//     ones), then H[r] += w_r D2[r][0..d-1] and s[r] += w_r D2[r][d] in fp32:
-//     the state is read and written once more, as 16-byte accesses.
+// Scores as a quadratic form. With U_a[m][b] = w_(a,b) [H | s][r(a, b)][m] for
+// b >= a (zero for b < a),
+//   phi(k)^T [H | s][:, m] = sum_a k[a] sum_b k[b] U_a[m][b],
+// so for every a one MMA D_a[c][m] = sum_b k_c[b] U_a[m][b] takes the bf16
+// candidate keys as they are (exact) and U_a split into two bf16 parts
+// (hi + lo, relative residual below 2^-16), and the epilogue accumulates
+// k_c[a] D_a[c][m] in fp32 registers. Every state value is converted once, and
+// the state streams from HBM once. The SRE is a distance of order |v|^2 and
+// keeps fp32-level accuracy (1e-7 relative on the synthetic candidates).
+//
+// Merge, 128 packed rows at a time: D2[r][e] = sum_m k_m[a_r] k_m[b_r]
+// [v_m | 1][e] with exact products (the product of two bf16 values splits
+// exactly into two bf16 parts), then H[r] += w_r D2[r][0..d-1] and
+// s[r] += w_r D2[r][d] in fp32.
+//
+// One CTA per head (bf16 candidates, d = 32 or 64, at most 256 of them), 18
+// warps: 16 workers (operand conversion and epilogues; warp w reads tensor-
+// memory lanes 32 (w % 4) ..), a producer warp (bulk copies of the state),
+// an MMA warp (one elected lane issues). Roles hand work over through
+// mbarrier rings; every wait is bounded.
 #include "kata_common.cuh"
 #include "kata_internal.h"
 #include "sm100.cuh"
@@ -37,275 +39,379 @@ namespace {
 using namespace sm100;
 using tc::warp_wait;
 
-constexpr int kST = 512;     // threads (16 warps)
-constexpr int kKR = 32;      // packed rows per score step (the MMA K extent)
-constexpr int kLR = 64;      // packed rows per staging copy
-constexpr int kStages = 3;   // staging copies in flight
-constexpr int kNMax = 256;   // candidates per head
-constexpr int kMR = 128;     // packed rows per merge tile
-constexpr int kMK = 32;      // merged candidates per merge step
+constexpr int kWorkers = 512;           // 16 worker warps
+constexpr int kThreads = kWorkers + 64;  // + producer warp + MMA warp
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kLR = 64;                 // packed rows per staging copy
+constexpr int kNMax = 256;              // candidates per head
+constexpr int kMR = 128;                // packed rows per merge tile
+constexpr int kMK = 32;                 // merged candidates per merge K chunk
+constexpr int kLag = 2;                 // the epilogue of a trails the build of a by this
+constexpr int kNB = 3;                  // U_a operand buffers
+constexpr int kND = 3;                  // D_a accumulators in tensor memory
+constexpr int kNA = 4;                  // merge operand buffers
+constexpr int kStSlots = 10;            // staging copies in flight, at most
+constexpr int kKmtPitch = 264;          // merged keys, transposed: row pitch (bank spread)
 constexpr float kSqrt2f = 1.41421356237309515f;
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in a K-major tile with
-// 64-byte rows (32 bf16 along K) under the 64-byte swizzle: chunk c of row r
-// is stored at chunk c ^ ((r >> 1) & 3). Tiles start on a 1024-byte boundary.
-__device__ __forceinline__ uint32_t sw64_chunk(int row, int chunk) {
-    return (uint32_t)(row * 64 + (((chunk ^ (row >> 1)) & 3) << 4));
+// K-major operand tiles with RB-byte rows (RB = 128: 128-byte swizzle, RB =
+// 64: 64-byte swizzle): byte offset of 16-byte chunk `chunk` of row `row`, and
+// the descriptor at K-step ks (16 elements, 32 bytes). Tiles start on a
+// 1024-byte boundary.
+template <int RB>
+__device__ __forceinline__ uint32_t kmaj_off(int row, int chunk) {
+    if constexpr (RB == 128)
+        return (uint32_t)(row * 128 + (((chunk ^ row) & 7) << 4));
+    else
+        return (uint32_t)(row * 64 + (((chunk ^ (row >> 1)) & 3) << 4));
 }
-// Descriptor of such a tile at K-step kk (16 elements, 32 bytes).
-__device__ __forceinline__ uint64_t kmaj64_desc(uint32_t base, int kk) {
-    return smem_desc(base + 32 * kk, 16, 512, kSwizzle64);
+template <int RB>
+__device__ __forceinline__ uint64_t kmaj_desc_rb(uint32_t base, int ks) {
+    return smem_desc(base + 32 * ks, 16, RB * 8, RB == 128 ? kSwizzle128 : kSwizzle64);
 }
-
-__device__ __forceinline__ uint32_t bf16_bits(float x) {
-    const __nv_bfloat16 b = __float2bfloat16_rn(x);
-    return (uint32_t)*reinterpret_cast<const uint16_t *>(&b);
-}
-__device__ __forceinline__ float bits_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
 // Eight values -> two 16-byte rows of bf16 parts, x = hi + lo (+ the residual
-// of a value with more than 16 significant bits).
+// of a value with more than 16 significant bits); pairs convert together.
 __device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
-    uint32_t h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        h[u] = bf16_bits(x[u]);
-        l[u] = bf16_bits(x[u] - bits_f32(h[u]));
+    for (int p = 0; p < 4; ++p) {
+        h[p] = pack_bf16x2(x[2 * p], x[2 * p + 1]);
+        l[p] = pack_bf16x2(x[2 * p] - __uint_as_float(h[p] << 16),
+                           x[2 * p + 1] - __uint_as_float(h[p] & 0xFFFF0000u));
     }
-    hi = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
-    lo = make_uint4(l[0] | (l[1] << 16), l[2] | (l[3] << 16), l[4] | (l[5] << 16), l[6] | (l[7] << 16));
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
+
+// The two bf16 values of a packed pair as fp32.
+__device__ __forceinline__ float lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __device__ __forceinline__ float row_weight(uint16_t ab) {
     return (ab >> 8) != (ab & 255) ? kSqrt2f : 1.f;
 }
 
+// 32 lanes x 8 or 1 consecutive 32-bit tensor-memory columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t &r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+
 enum SreBar {
-    kBLoad = 0,                 // kStages: a staging copy landed
-    kBMma = kBLoad + kStages,   // 2: the score MMAs reading operand buffer i completed
-    kBFinal = kBMma + 2,        // every score MMA completed
-    kBM2 = kBFinal + 1,         // 2: the merge MMAs reading operand buffer i completed
-    kBDrain = kBM2 + 2,         // teardown: every MMA completed
-    kBCount = kBDrain + 1
+    kStFull = 0,                     // kStSlots: a staging copy landed (tx count)
+    kStEmpty = kStFull + kStSlots,   // kStSlots: every worker warp is done with a copy
+    kBbFull = kStEmpty + kStSlots,   // kNB: U_a written (worker warps)
+    kBbEmpty = kBbFull + kNB, // kNB: the MMAs reading U_a completed
+    kDFull = kBbEmpty + kNB,  // kND: D_a complete
+    kDEmpty = kDFull + kND,   // kND: D_a read (worker warps)
+    kA2Full = kDEmpty + kND,  // kNA: a merge operand chunk written
+    kA2Empty = kA2Full + kNA, // kNA: the MMAs reading it completed
+    kD2Full = kA2Empty + kNA, // 2: a merge tile's D2 complete
+    kD2Empty = kD2Full + 2,   // 2: D2 read (worker warps)
+    kDrain = kD2Empty + 2,    // teardown: every MMA completed
+    kBarCount = kDrain + 1
 };
 
 template <int DH>
 struct SreCfg {
     static constexpr int D = DH * (DH + 1) / 2;
-    static constexpr int N2 = DH + 16;                       // merge MMA N: [v | 1 | 0]
+    static constexpr int RB = 2 * DH;           // K-major rows of DH bf16
+    static constexpr int KS = DH / 16;          // K-steps over b
+    static constexpr int NCH = DH / 8;          // 16-byte chunks per row
+    static constexpr int N1 = DH + 16;          // score MMA N: [H | s | 0] columns
+    static constexpr int N2 = DH + 16;          // merge MMA N: [v | 1 | 0]
+    static constexpr int EC = DH / 4;           // epilogue columns per worker warp
+    static constexpr int NST = DH == 64 ? 6 : 10;
+    static constexpr int NL = (D + kLR - 1) / kLR;  // staging copies
     static constexpr int STG = ((kLR * DH + kLR) * 4 + 1023) / 1024 * 1024;
-    static constexpr int ATILE = 128 * 64;                   // 128 rows x 32 bf16
-    static constexpr int BTILE = kNMax * 64;                 // 256 rows x 32 bf16
-    static constexpr int B2TILE = N2 * 64;                   // a multiple of 1024
-    static constexpr int OFF_STG = 0;                        // phase 3: k of merged [256][DH]
-    static constexpr int OFF_A = OFF_STG + kStages * STG;    // [2 buffers][hi, lo]
-    static constexpr int OFF_B = OFF_A + 2 * 2 * ATILE;      // [2 buffers][hi, lo]; phase 3: B2
-    static constexpr int OFF_KT = OFF_B + 2 * 2 * BTILE;     // k^T [DH][256] bf16
-    static constexpr int OFF_TAB = OFF_KT + DH * kNMax * 2;  // pair of each packed row
+    static constexpr int KA_BYTES = kNMax * RB;
+    static constexpr int BPART = (N1 * RB + 1023) / 1024 * 1024;
+    static constexpr int A2PART = kMR * 64;
+    static constexpr int B2TILE = N2 * 64;
+    static constexpr int OFF_KA = 0;
+    static constexpr int OFF_STG = OFF_KA + KA_BYTES;
+    static constexpr int OFF_BB = OFF_STG + NST * STG;  // [kNB][hi, lo]
+    static constexpr int OFF_B2 = OFF_STG;              // merge: over the staging copies
+    static constexpr int OFF_A2 = OFF_B2 + (kNMax / kMK) * B2TILE;  // [kNA][hi, lo]
+    static constexpr int OFF_KMT = OFF_A2 + kNA * 2 * A2PART;  // merge: keys [DH][kKmtPitch]
+    static constexpr int OFF_TAB = OFF_BB + kNB * 2 * BPART;
     static constexpr int OFF_SC = OFF_TAB + (D * 2 + 15) / 16 * 16;
-    static constexpr int OFF_BAR = OFF_SC + 5 * kNMax * 4;   // five per-candidate arrays
-    static constexpr int BYTES = OFF_BAR + kBCount * 8 + 16 + 1024;
-    static_assert(B2TILE % 1024 == 0, "merge operand tiles stay 1024-aligned");
-    static_assert(8 * B2TILE <= 2 * 2 * BTILE, "merge operand fits the score operand area");
-    static_assert(kNMax * (DH + 1) * 4 <= 2 * 2 * (ATILE + BTILE), "squared errors fit");
-    static_assert(kNMax * DH * 2 <= kStages * STG, "merged keys fit the staging area");
+    static constexpr int OFF_BAR = OFF_SC + 9 * kNMax * 4;  // 5 arrays + 4 partial sums
+    static constexpr int BYTES = OFF_BAR + kBarCount * 8 + 16 + 1024;
+    static_assert(NST <= kStSlots, "barrier slots");
+    static_assert(B2TILE % 1024 == 0 && BPART % 1024 == 0 && STG % 1024 == 0, "alignment");
+    static_assert(OFF_KMT + DH * kKmtPitch * 2 <= OFF_TAB, "merge operands fit");
     static_assert(BYTES <= 227 * 1024, "shared memory");
+    static_assert(kND * 2 * N1 <= 512 && 128 + N2 <= 512, "tensor memory");
 };
 
 template <int DH>
-__global__ void __launch_bounds__(kST, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict__ kc,
               const __nv_bfloat16 *__restrict__ vc, long cand_head_stride,
               const int *__restrict__ pos, long pos_head_stride, int n, int keep, float eps,
               int merge, float *__restrict__ scores, int *__restrict__ keep_idx,
               float *Hst_mut, float *s_mut, unsigned int *errw) {
     using L = SreCfg<DH>;
-    constexpr int D = L::D;
-    constexpr int NCH = (D + kKR - 1) / kKR;  // score steps
-    constexpr int NL = (D + kLR - 1) / kLR;   // staging copies
-    constexpr int N2 = L::N2;
+    constexpr int D = L::D, RB = L::RB, N1 = L::N1, N2 = L::N2, EC = L::EC, NST = L::NST;
+    constexpr int NL = L::NL;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_BAR + kBCount * 8);
-    uint16_t *kT = reinterpret_cast<uint16_t *>(sm + L::OFF_KT);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_BAR + kBarCount * 8);
+    uint8_t *KA = sm + L::OFF_KA;
     uint16_t *tab = reinterpret_cast<uint16_t *>(sm + L::OFF_TAB);
     float *sc = reinterpret_cast<float *>(sm + L::OFF_SC);
     float *den = sc + kNMax;
     int *cpos = reinterpret_cast<int *>(den + kNMax);
     int *kflag = cpos + kNMax;
     int *mlist = kflag + kNMax;
+    float *sqp = reinterpret_cast<float *>(mlist + kNMax);  // [4][256]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x;
-    const int NP = (n + 15) & ~15;  // score MMA N: candidates padded to 16
+    const int nmt = n > 128 ? 2 : 1;  // 128-candidate M tiles
     const ErrCtx err{errw};
     const float *Hh = Hst + (size_t)h * D * DH;
     const float *sh = s + (size_t)h * D;
     const __nv_bfloat16 *kh = kc + (size_t)h * cand_head_stride;
     const __nv_bfloat16 *vh = vc + (size_t)h * cand_head_stride;
+    const bool worker = warp < kProducerWarp;
+    const int qd = warp & 3, g = (warp >> 2) & 3;  // worker: lane quadrant, column group
+    const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
+    // ---------------- set-up ----------------
     if (tid == 0) {
-        for (int i = 0; i < kBCount; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&bar[kStFull + i], 1);
+            mbar_init(&bar[kStEmpty + i], 16);
+        }
+        for (int i = 0; i < kNB; ++i) {
+            mbar_init(&bar[kBbFull + i], 16);
+            mbar_init(&bar[kBbEmpty + i], 1);
+        }
+        for (int i = 0; i < kND; ++i) {
+            mbar_init(&bar[kDFull + i], 1);
+            mbar_init(&bar[kDEmpty + i], 16);
+        }
+        for (int i = 0; i < kNA; ++i) {
+            mbar_init(&bar[kA2Full + i], 16);
+            mbar_init(&bar[kA2Empty + i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar[kD2Full + i], 1);
+            mbar_init(&bar[kD2Empty + i], 16);
+        }
+        mbar_init(&bar[kDrain], 1);
         cta_abort_clear();
         fence_barrier_init();
     }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    int issued = 0;  // staging copies issued (thread 0)
-    auto issue_load = [&](int j) {
-        const int r0 = j * kLR, rows = D - r0 < kLR ? D - r0 : kLR;
-        uint8_t *dst = sm + L::OFF_STG + (j % kStages) * L::STG;
-        const uint32_t hb = (uint32_t)(rows * DH * 4), sb = (uint32_t)(rows * 4);
-        mbar_arrive_expect_tx(&bar[kBLoad + j % kStages], hb + sb);
-        bulk_load(dst, Hh + (size_t)r0 * DH, hb, &bar[kBLoad + j % kStages]);
-        bulk_load(dst + kLR * DH * 4, sh + r0, sb, &bar[kBLoad + j % kStages]);
-        ++issued;
-    };
-    __syncthreads();  // barriers initialised
-    if (tid == 0)
-        for (int j = 0; j < kStages && j < NL; ++j) issue_load(j);
-    // pair table; k^T with zeros past n; rows d+1 .. 127 of the A operands are
-    // zero in both buffers and both parts
-    for (int r = tid; r < D; r += kST) {
-        int a = 0;
-        while (packed_row_base(a + 1, DH) <= r) ++a;
-        tab[r] = (uint16_t)((a << 8) | (a + r - packed_row_base(a, DH)));
-    }
-    for (int idx = tid; idx < kNMax * DH; idx += kST) {
-        const int c = idx / DH, a = idx % DH;
-        kT[a * kNMax + c] = c < n ? reinterpret_cast<const uint16_t *>(kh)[(size_t)c * DH + a] : 0;
-    }
-    {
-        constexpr int z0 = (DH + 1) * 64, zq = (L::ATILE - z0) / 16;
-        for (int idx = tid; idx < 4 * zq; idx += kST)
-            *reinterpret_cast<uint4 *>(sm + L::OFF_A + (idx / zq) * L::ATILE + z0 +
-                                       (idx % zq) * 16) = make_uint4(0, 0, 0, 0);
+    build_pair_table(tab, DH);
+    if (worker) {
+        // candidate keys as the score MMA's A operand (zero rows past n)
+        for (int idx = tid; idx < nmt * 128 * L::NCH; idx += kWorkers) {
+            const int c = idx / L::NCH, ch = idx % L::NCH;
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (c < n) x = *reinterpret_cast<const uint4 *>(kh + (size_t)c * DH + ch * 8);
+            *reinterpret_cast<uint4 *>(KA + kmaj_off<RB>(c, ch)) = x;
+        }
+        // rows DH + 1 .. N1 - 1 of every U_a buffer and part stay zero
+        constexpr int zrows = N1 - DH - 1;
+        for (int idx = tid; idx < kNB * 2 * zrows * L::NCH; idx += kWorkers) {
+            const int part = idx / (zrows * L::NCH), rem = idx % (zrows * L::NCH);
+            const int row = DH + 1 + rem / L::NCH, ch = rem % L::NCH;
+            *reinterpret_cast<uint4 *>(sm + L::OFF_BB + part * L::BPART + kmaj_off<RB>(row, ch)) =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    bool ok = true;
+    int issued = 0;  // staging copies issued (producer warp)
 
     // ---------------- 1. scores ----------------
-    const uint32_t id_s = idesc_bf16(128, NP, 0, 0);
-    bool ok = true;
-    for (int i = 0; i < NCH; ++i) {
-        const int j = i >> 1, half = i & 1, buf = i & 1;
-        const float *stg = reinterpret_cast<const float *>(sm + L::OFF_STG + (j % kStages) * L::STG);
-        uint8_t *Ah = sm + L::OFF_A + buf * 2 * L::ATILE, *Al = Ah + L::ATILE;
-        uint8_t *Bh = sm + L::OFF_B + buf * 2 * L::BTILE, *Bl = Bh + L::BTILE;
-        // this step's rows have landed; the MMAs of step i - 2 (the last
-        // readers of operand buffer buf) have completed
-        ok = warp_wait(&bar[kBLoad + j % kStages], (j / kStages) & 1, err, 0x701) && ok;
-        if (i >= 2) ok = warp_wait(&bar[kBMma + buf], ((i - 2) >> 1) & 1, err, 0x702) && ok;
-        // A: row m (a value column, or the normaliser at m = DH), 8 packed rows
-        // per task
-        for (int idx = tid; idx < 4 * (DH + 1); idx += kST) {
-            const int m = idx < 4 * DH ? idx % DH : DH;
-            const int kg = idx < 4 * DH ? idx / DH : idx - 4 * DH;
-            float x[8];
+    float acc[2][EC];
+    float sacc[2] = {0.f, 0.f};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int rr = kg * 8 + u, r = i * kKR + rr, lr = half * kKR + rr;
-                x[u] = r < D ? row_weight(tab[r]) * (m < DH ? stg[lr * DH + m] : stg[kLR * DH + lr])
-                             : 0.f;
-            }
-            uint4 hi, lo;
-            split8(x, hi, lo);
-            *reinterpret_cast<uint4 *>(Ah + sw64_chunk(m, kg)) = hi;
-            *reinterpret_cast<uint4 *>(Al + sw64_chunk(m, kg)) = lo;
-        }
-        // B: row c (a candidate), 8 packed rows of k_c[a] k_c[b] per task
-        for (int idx = tid; idx < 4 * NP; idx += kST) {
-            const int c = idx % NP, kg = idx / NP;
-            float x[8];
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = i * kKR + kg * 8 + u;
-                float p = 0.f;
-                if (r < D) {
-                    const int ab = tab[r];
-                    p = bits_f32(kT[(ab >> 8) * kNMax + c]) * bits_f32(kT[(ab & 255) * kNMax + c]);
-                }
-                x[u] = p;
-            }
-            uint4 hi, lo;
-            split8(x, hi, lo);
-            *reinterpret_cast<uint4 *>(Bh + sw64_chunk(c, kg)) = hi;
-            *reinterpret_cast<uint4 *>(Bl + sw64_chunk(c, kg)) = lo;
-        }
-        fence_proxy_async_smem();
-        ok = bar_sync_and(1, kST, ok);
-        if (!ok) break;
-        if (tid == 0) {
-            // both halves of staging copy j are converted: refill its buffer
-            if (half == 1 && j + kStages < NL) issue_load(j + kStages);
-            tc_fence_after();
-            const uint32_t ah = smem_u32(Ah), al = smem_u32(Al);
-            const uint32_t bh = smem_u32(Bh), bl = smem_u32(Bl);
-#pragma unroll
-            for (int kk = 0; kk < kKR / 16; ++kk) {
-                mma_ss(tmem, kmaj64_desc(ah, kk), kmaj64_desc(bh, kk), id_s, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_ss(tmem, kmaj64_desc(ah, kk), kmaj64_desc(bl, kk), id_s, 1u);
-                mma_ss(tmem, kmaj64_desc(al, kk), kmaj64_desc(bh, kk), id_s, 1u);
-            }
-            mma_commit(&bar[kBMma + buf]);
-        }
-    }
-    if (tid == 0) mma_commit(&bar[kBFinal]);
-    ok = warp_wait(&bar[kBFinal], 0, err, 0x703) && ok;
-    tc_fence_after();
-    ok = bar_sync_and(1, kST, ok);
+        for (int i = 0; i < EC; ++i) acc[mt][i] = 0.f;
 
-    // ---------------- 2. SRE and the kept set ----------------
-    const int m_keep = keep < n ? keep : n;
-    const int nm = n - m_keep;
-    if (ok) {
-        if (warp == DH / 32) {  // tensor-memory lane DH: the normaliser of every candidate
-            for (int c0 = 0; c0 < NP; c0 += 16) {
-                uint32_t r16[16];
-                tmem_ld16(tmem + lane_base + c0, r16);
-                tmem_ld_wait();
-                if (lane == 0)
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) den[c0 + u] = __uint_as_float(r16[u]);
+    if (warp == kProducerWarp) {
+        for (int st = 0; st < NL; ++st) {
+            const int slot = st % NST, use = st / NST;
+            if (use >= 1) ok = warp_wait(&bar[kStEmpty + slot], (use - 1) & 1, err, 0x711) && ok;
+            if (!ok) break;
+            if (lane == 0) {
+                const int r0 = st * kLR, rows = D - r0 < kLR ? D - r0 : kLR;
+                uint8_t *dst = sm + L::OFF_STG + slot * L::STG;
+                const uint32_t hb = (uint32_t)(rows * DH * 4), sb = (uint32_t)(rows * 4);
+                mbar_arrive_expect_tx(&bar[kStFull + slot], hb + sb);
+                bulk_load(dst, Hh + (size_t)r0 * DH, hb, &bar[kStFull + slot]);
+                bulk_load(dst + kLR * DH * 4, sh + r0, sb, &bar[kStFull + slot]);
             }
+            ++issued;
+            __syncwarp();
         }
-        __syncthreads();
-        // squared differences, one value column per thread of warps 0 .. DH/32 - 1,
-        // staged as sq[c][e] (pitch DH + 1) over the free operand buffers
-        float *sq = reinterpret_cast<float *>(sm + L::OFF_A);
-        if (warp < DH / 32) {
-            const int e = tid;
-            for (int c0 = 0; c0 < NP; c0 += 16) {
-                uint32_t r16[16];
-                tmem_ld16(tmem + lane_base + c0, r16);
-                tmem_ld_wait();
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int c = c0 + u;
-                    if (c < n) {
-                        const float diff = __uint_as_float(r16[u]) / (den[c] + eps) -
-                                           __bfloat162float(vh[(size_t)c * DH + e]);
-                        sq[c * (DH + 1) + e] = diff * diff;
+    } else if (warp == kMmaWarp) {
+        const uint32_t id1 = idesc_bf16(128, N1, 0, 0);
+        for (int a = 0; a < DH; ++a) {
+            const int i = a % kNB, j = a % kND;
+            ok = warp_wait(&bar[kBbFull + i], (a / kNB) & 1, err, 0x712) && ok;
+            if (a >= kND) ok = warp_wait(&bar[kDEmpty + j], ((a / kND) - 1) & 1, err, 0x713) && ok;
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t bh = smem_u32(sm + L::OFF_BB + i * 2 * L::BPART), bl = bh + L::BPART;
+                const int ks0 = a / 16;
+                for (int mt = 0; mt < nmt; ++mt) {
+                    const uint32_t d = tmem + (uint32_t)((j * nmt + mt) * N1);
+                    const uint32_t ka = smem_u32(KA + mt * 128 * RB);
+                    for (int ks = ks0; ks < L::KS; ++ks) {
+                        mma_ss(d, kmaj_desc_rb<RB>(ka, ks), kmaj_desc_rb<RB>(bh, ks), id1,
+                               ks > ks0 ? 1u : 0u);
+                        mma_ss(d, kmaj_desc_rb<RB>(ka, ks), kmaj_desc_rb<RB>(bl, ks), id1, 1u);
                     }
                 }
+                mma_commit(&bar[kBbEmpty + i]);
+                mma_commit(&bar[kDFull + j]);
+            }
+            __syncwarp();
+        }
+    } else {
+        int waited = 0, released = 0;  // staging copies waited for / released (warp-uniform)
+        uint4 kreg[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        for (int it = 0; it < DH + kLag && ok; ++it) {
+            if (it < DH) {  // U_it: rows m (value columns and the normaliser), K = b
+                const int a = it, i = a % kNB;
+                const int first = packed_row_base(a, DH), last = first + DH - 1 - a;
+                while (waited <= last / kLR && ok) {
+                    ok = warp_wait(&bar[kStFull + waited % NST], (waited / NST) & 1, err, 0x714) && ok;
+                    ++waited;
+                }
+                if (a >= kNB) ok = warp_wait(&bar[kBbEmpty + i], ((a / kNB) - 1) & 1, err, 0x715) && ok;
+                if (!ok) break;
+                uint8_t *Bh = sm + L::OFF_BB + i * 2 * L::BPART, *Bl = Bh + L::BPART;
+                const int ch0 = (a / 16) * 2, ntask = (DH + 1) * (L::NCH - ch0);
+                for (int idx = tid; idx < ntask; idx += kWorkers) {
+                    const int m = idx % (DH + 1), ch = ch0 + idx / (DH + 1);
+                    // rows of b = 8 ch .. 8 ch + 7 (those with b < a are zero):
+                    // consecutive packed rows, in at most two staging copies
+                    const int b0 = ch * 8, rs = first + (b0 > a ? b0 - a : 0);
+                    const int st0 = rs / kLR;
+                    const float *p0 = reinterpret_cast<const float *>(sm + L::OFF_STG + (st0 % NST) * L::STG);
+                    const float *p1 = reinterpret_cast<const float *>(sm + L::OFF_STG + ((st0 + 1) % NST) * L::STG);
+                    const int col = m < DH ? m : kLR * DH;  // value column, or the normaliser
+                    const int rstride = m < DH ? DH : 1;
+                    float x[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int b = b0 + u, bb = b > a ? b : a;  // rows b < a are not read
+                        const int lr = first + bb - a - st0 * kLR;  // row inside copy st0 (or past it)
+                        const float *pp = lr < kLR ? p0 + lr * rstride : p1 + (lr - kLR) * rstride;
+                        const float val = pp[col];
+                        x[u] = b > a ? kSqrt2f * val : (b == a ? val : 0.f);
+                    }
+                    uint4 hi, lo;
+                    split8(x, hi, lo);
+                    *reinterpret_cast<uint4 *>(Bh + kmaj_off<RB>(m, ch)) = hi;
+                    *reinterpret_cast<uint4 *>(Bl + kmaj_off<RB>(m, ch)) = lo;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kBbFull + i]);
+                // staging copies whose rows all come before the next index
+                const int lim = a == DH - 1 ? NL : packed_row_base(a + 1, DH) / kLR;
+                for (; released < lim; ++released)
+                    if (lane == 0) mbar_arrive(&bar[kStEmpty + released % NST]);
+            }
+            if (it >= kLag) {  // acc += k_c[a] D_a[c][columns of this warp]
+                const int a = it - kLag, j = a % kND;
+                ok = warp_wait(&bar[kDFull + j], (a / kND) & 1, err, 0x716) && ok;
+                if (!ok) break;
+                tc_fence_after();
+                if ((a & 7) == 0) {  // this thread's candidates' keys a .. a + 7
+                    kreg[0] = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(qd * 32 + lane, a >> 3));
+                    if (nmt > 1)
+                        kreg[1] = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(128 + qd * 32 + lane, a >> 3));
+                }
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    if (mt >= nmt) break;
+                    const uint32_t col = (uint32_t)((j * nmt + mt) * N1);
+                    uint32_t v[EC], sv = 0u;
+                    if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
+                    else tmem_ld8(tmem + lane_base + col + EC * g, v);
+                    if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
+                    tmem_ld_wait();
+                    const uint4 k4 = kreg[mt];
+                    const uint32_t kw = (a & 4) ? ((a & 2) ? k4.w : k4.z) : ((a & 2) ? k4.y : k4.x);
+                    const float kca = (a & 1) ? hi_f32(kw) : lo_f32(kw);
+#pragma unroll
+                    for (int u = 0; u < EC; ++u)
+                        acc[mt][u] = fmaf(kca, __uint_as_float(v[u]), acc[mt][u]);
+                    sacc[mt] = fmaf(kca, __uint_as_float(sv), sacc[mt]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kDEmpty + j]);
             }
         }
-        tc_fence_before();
-        __syncthreads();
+    }
+    ok = bar_sync_and(0, kThreads, ok);
+
+    // ---------------- 2. SRE and the kept set (workers) ----------------
+    const int m_keep = keep < n ? keep : n;
+    const int nm = n - m_keep;
+    if (ok && worker) {
+        if (g == 0) {
+            den[qd * 32 + lane] = sacc[0];
+            if (nmt > 1) den[128 + qd * 32 + lane] = sacc[1];
+        }
+        bar_sync_and(1, kWorkers, true);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            const int c = mt * 128 + qd * 32 + lane;
+            if (mt < nmt && c < n) {
+                const float inv_den = 1.f / (den[c] + eps);
+                const uint4 *vr = reinterpret_cast<const uint4 *>(vh + (size_t)c * DH + EC * g);
+                float part = 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < EC / 8; ++q4) {
+                    const uint4 w4 = vr[q4];
+                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float vv = (u & 1) ? hi_f32(wv[u >> 1]) : lo_f32(wv[u >> 1]);
+                        const float diff = acc[mt][q4 * 8 + u] * inv_den - vv;
+                        part = fmaf(diff, diff, part);
+                    }
+                }
+                sqp[g * kNMax + c] = part;
+            }
+        }
+        bar_sync_and(1, kWorkers, true);
         if (tid < n) {
-            float acc = 0.f;
-            for (int e = 0; e < DH; ++e) acc += sq[tid * (DH + 1) + e];
-            sc[tid] = isnan(acc) ? -INFINITY : acc;  // a total order even for 0/0 scores
+            const float e2 = (sqp[tid] + sqp[kNMax + tid]) + (sqp[2 * kNMax + tid] + sqp[3 * kNMax + tid]);
+            sc[tid] = isnan(e2) ? -INFINITY : e2;  // a total order even for 0/0 scores
             cpos[tid] = pos[(size_t)h * pos_head_stride + tid];
             if (scores) scores[(size_t)h * n + tid] = sc[tid];
         }
-        __syncthreads();
+        bar_sync_and(1, kWorkers, true);
         if (tid < n) {
             const float si = sc[tid];
             const int pi = cpos[tid];
@@ -317,7 +423,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
             }
             kflag[tid] = rank < m_keep;
         }
-        __syncthreads();
+        bar_sync_and(1, kWorkers, true);
         if (tid < n) {
             const int pi = cpos[tid];
             if (kflag[tid]) {
@@ -331,135 +437,168 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                 mlist[mr] = tid;
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
 
     // ---------------- 3. merge ----------------
     if (ok && merge && nm > 0) {
         const int nk2 = (nm + kMK - 1) / kMK;
         constexpr int NT2 = (D + kMR - 1) / kMR;
-        // keys of the merged candidates, row-major [mi][DH], zero past nm
-        uint16_t *kM = reinterpret_cast<uint16_t *>(sm + L::OFF_STG);
-        for (int idx = tid; idx < nk2 * kMK * DH; idx += kST) {
-            const int mi = idx / DH, a = idx % DH;
-            kM[idx] = mi < nm ? reinterpret_cast<const uint16_t *>(kh)[(size_t)mlist[mi] * DH + a] : 0;
-        }
-        // B2 (K-major), step q: row e < DH is v[e] of merged candidates
-        // 32 q .. 32 q + 31, row DH is 1, rows above are 0 (zero past nm)
-        uint8_t *B2 = sm + L::OFF_B;
-        for (int idx = tid; idx < nk2 * N2 * 4; idx += kST) {
-            const int q = idx / (N2 * 4), rem = idx % (N2 * 4);
-            const int kg = rem / N2, e = rem % N2;
-            uint32_t b[8];
+        uint8_t *B2 = sm + L::OFF_B2;
+        if (warp == kMmaWarp) {
+            const uint32_t id2 = idesc_bf16(128, N2, 0, 0);
+            for (int t = 0; t < NT2 && ok; ++t) {
+                for (int q = 0; q < nk2; ++q) {
+                    const int ci = t * nk2 + q, slot = ci % kNA;
+                    ok = warp_wait(&bar[kA2Full + slot], (ci / kNA) & 1, err, 0x721) && ok;
+                    if (q == 0 && t >= 2)
+                        ok = warp_wait(&bar[kD2Empty + (t & 1)], ((t >> 1) - 1) & 1, err, 0x722) && ok;
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t d2 = tmem + (uint32_t)((t & 1) * 128);
+                        const uint32_t ah = smem_u32(sm + L::OFF_A2 + slot * 2 * L::A2PART);
+                        const uint32_t al = ah + L::A2PART;
+                        const uint32_t b2 = smem_u32(B2 + q * L::B2TILE);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int mi = q * kMK + kg * 8 + u;
-                uint32_t val = 0;
-                if (mi < nm) {
-                    if (e < DH)
-                        val = reinterpret_cast<const uint16_t *>(vh)[(size_t)mlist[mi] * DH + e];
-                    else if (e == DH)
-                        val = 0x3F80u;  // 1.0 in bf16
+                        for (int kk = 0; kk < kMK / 16; ++kk) {
+                            mma_ss(d2, kmaj_desc_rb<64>(ah, kk), kmaj_desc_rb<64>(b2, kk), id2,
+                                   (q > 0 || kk > 0) ? 1u : 0u);
+                            mma_ss(d2, kmaj_desc_rb<64>(al, kk), kmaj_desc_rb<64>(b2, kk), id2, 1u);
+                        }
+                        mma_commit(&bar[kA2Empty + slot]);
+                        if (q == nk2 - 1) mma_commit(&bar[kD2Full + (t & 1)]);
+                    }
+                    __syncwarp();
                 }
-                b[u] = val;
             }
-            *reinterpret_cast<uint4 *>(B2 + q * L::B2TILE + sw64_chunk(e, kg)) =
-                make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16),
-                           b[6] | (b[7] << 16));
-        }
-        __syncthreads();  // the merged keys are read by other threads below
-        const uint32_t id_m = idesc_bf16(128, N2, 0, 0);
-        // epilogue share of each thread: tile row 32 (warp % 4) + lane, the
-        // column group warp / 4 (16 columns at DH = 64, 8 at 32)
-        constexpr int EC = DH / 4;
-        const int cg = warp >> 2;
-        float4 hreg[EC / 4];
-        float sreg = 0.f;
-        const int nsteps = NT2 * nk2;
-        for (int st = 0; st < nsteps; ++st) {
-            const int t = st / nk2, q = st % nk2, buf = st & 1;
-            const int row = t * kMR + (warp & 3) * 32 + lane;
-            if (q == 0 && row < D) {  // this tile's state, read early
-                const float4 *src = reinterpret_cast<const float4 *>(Hh + (size_t)row * DH + cg * EC);
-#pragma unroll
-                for (int u = 0; u < EC / 4; ++u) hreg[u] = src[u];
-                if (cg == 0) sreg = sh[row];
-            }
-            uint8_t *Ah = sm + L::OFF_A + buf * 2 * L::ATILE, *Al = Ah + L::ATILE;
-            if (st >= 2) ok = warp_wait(&bar[kBM2 + buf], ((st - 2) >> 1) & 1, err, 0x704) && ok;
-            {   // A2: tile row rr, merged candidates 32 q + 8 kg .. +7 (kg warp-uniform)
-                const int rr = tid & 127, kg = tid >> 7;
-                const int r = t * kMR + rr;
-                float x[8];
-                int a = 0, b = 0;
-                if (r < D) {
-                    const int ab = tab[r];
-                    a = ab >> 8;
-                    b = ab & 255;
-                }
+        } else if (worker) {
+            // B2 (K-major), chunk q: row e < DH is v[e] of merged candidates
+            // 32 q .. 32 q + 31, row DH is 1, rows above are 0 (zero past nm)
+            for (int idx = tid; idx < nk2 * N2 * 4; idx += kWorkers) {
+                const int q = idx / (N2 * 4), rem = idx % (N2 * 4);
+                const int kg = rem / N2, e = rem % N2;
+                uint32_t bv[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int mi = q * kMK + kg * 8 + u;
-                    x[u] = r < D ? bits_f32(kM[mi * DH + a]) * bits_f32(kM[mi * DH + b]) : 0.f;
-                }
-                uint4 hi, lo;
-                split8(x, hi, lo);
-                *reinterpret_cast<uint4 *>(Ah + sw64_chunk(rr, kg)) = hi;
-                *reinterpret_cast<uint4 *>(Al + sw64_chunk(rr, kg)) = lo;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            ok = bar_sync_and(1, kST, ok);
-            if (!ok) break;
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t ah = smem_u32(Ah), al = smem_u32(Al);
-                const uint32_t b2 = smem_u32(B2 + q * L::B2TILE);
-#pragma unroll
-                for (int kk = 0; kk < kMK / 16; ++kk) {
-                    mma_ss(tmem, kmaj64_desc(ah, kk), kmaj64_desc(b2, kk), id_m, (q > 0 || kk > 0) ? 1u : 0u);
-                    mma_ss(tmem, kmaj64_desc(al, kk), kmaj64_desc(b2, kk), id_m, 1u);
-                }
-                mma_commit(&bar[kBM2 + buf]);
-            }
-            if (q == nk2 - 1) {  // H[r] += w_r D2[r], s[r] += w_r D2[r][DH]
-                ok = warp_wait(&bar[kBM2 + buf], (st >> 1) & 1, err, 0x705) && ok;
-                tc_fence_after();
-                uint32_t v16[16], s16[16];
-                tmem_ld16(tmem + lane_base + cg * EC, v16);
-                if (cg == 0) tmem_ld16(tmem + lane_base + DH, s16);
-                tmem_ld_wait();
-                if (ok && row < D) {
-                    const float w = row_weight(tab[row]);
-                    float4 *dst = reinterpret_cast<float4 *>(Hst_mut + ((size_t)h * D + row) * DH + cg * EC);
-#pragma unroll
-                    for (int u = 0; u < EC / 4; ++u) {
-                        float4 x = hreg[u];
-                        x.x = fmaf(w, __uint_as_float(v16[4 * u + 0]), x.x);
-                        x.y = fmaf(w, __uint_as_float(v16[4 * u + 1]), x.y);
-                        x.z = fmaf(w, __uint_as_float(v16[4 * u + 2]), x.z);
-                        x.w = fmaf(w, __uint_as_float(v16[4 * u + 3]), x.w);
-                        dst[u] = x;
+                    uint32_t val = 0;
+                    if (mi < nm) {
+                        if (e < DH)
+                            val = reinterpret_cast<const uint16_t *>(vh)[(size_t)mlist[mi] * DH + e];
+                        else if (e == DH)
+                            val = 0x3F80u;  // 1.0 in bf16
                     }
-                    if (cg == 0) s_mut[(size_t)h * D + row] = fmaf(w, __uint_as_float(s16[0]), sreg);
+                    bv[u] = val;
                 }
-                tc_fence_before();
+                *reinterpret_cast<uint4 *>(B2 + q * L::B2TILE + kmaj_off<64>(e, kg)) =
+                    make_uint4(bv[0] | (bv[1] << 16), bv[2] | (bv[3] << 16),
+                               bv[4] | (bv[5] << 16), bv[6] | (bv[7] << 16));
+            }
+            // merged keys, transposed: kmT[a][mi] (zero past nm)
+            uint16_t *kmT = reinterpret_cast<uint16_t *>(sm + L::OFF_KMT);
+            for (int idx = tid; idx < L::NCH * nk2 * kMK; idx += kWorkers) {
+                const int mi = idx % (nk2 * kMK), a8 = idx / (nk2 * kMK);
+                uint4 x = make_uint4(0, 0, 0, 0);
+                if (mi < nm) x = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(mlist[mi], a8));
+                const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    kmT[(a8 * 8 + u) * kKmtPitch + mi] = (uint16_t)(xw[u >> 1] >> ((u & 1) * 16));
+            }
+            bar_sync_and(1, kWorkers, true);
+            float4 hreg[EC / 4];
+            float sreg = 0.f;
+            for (int it = 0; it <= NT2 && ok; ++it) {
+                const int row = (it - 1) * kMR + qd * 32 + lane;  // epilogue row (tile it - 1)
+                if (it >= 1 && row < D) {  // read early, used after this iteration's build
+                    const float4 *src = reinterpret_cast<const float4 *>(Hh + (size_t)row * DH + EC * g);
+#pragma unroll
+                    for (int u = 0; u < EC / 4; ++u) hreg[u] = src[u];
+                    if (g == 0) sreg = sh[row];
+                }
+                if (it < NT2) {
+                    for (int q = 0; q < nk2; ++q) {
+                        const int ci = it * nk2 + q, slot = ci % kNA;
+                        if (ci >= kNA)
+                            ok = warp_wait(&bar[kA2Empty + slot], ((ci / kNA) - 1) & 1, err, 0x723) && ok;
+                        if (!ok) break;
+                        uint8_t *Ah = sm + L::OFF_A2 + slot * 2 * L::A2PART, *Al = Ah + L::A2PART;
+                        // tile row rr, merged candidates 32 q + 8 kg .. +7 (kg warp-uniform)
+                        const int rr = tid & 127, kg = tid >> 7;
+                        const int r = it * kMR + rr;
+                        float x[8];
+                        if (r < D) {
+                            const int ab = tab[r], col = q * kMK + kg * 8;
+                            const uint4 ka = *reinterpret_cast<const uint4 *>(kmT + (ab >> 8) * kKmtPitch + col);
+                            const uint4 kb = *reinterpret_cast<const uint4 *>(kmT + (ab & 255) * kKmtPitch + col);
+                            const uint32_t aw[4] = {ka.x, ka.y, ka.z, ka.w}, bw[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+                            for (int p = 0; p < 4; ++p) {
+                                x[2 * p] = lo_f32(aw[p]) * lo_f32(bw[p]);
+                                x[2 * p + 1] = hi_f32(aw[p]) * hi_f32(bw[p]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) x[u] = 0.f;
+                        }
+                        uint4 hi, lo;
+                        split8(x, hi, lo);
+                        *reinterpret_cast<uint4 *>(Ah + kmaj_off<64>(rr, kg)) = hi;
+                        *reinterpret_cast<uint4 *>(Al + kmaj_off<64>(rr, kg)) = lo;
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar[kA2Full + slot]);
+                    }
+                    if (!ok) break;
+                }
+                if (it >= 1) {  // H[r] += w_r D2[r], s[r] += w_r D2[r][DH]
+                    const int t = it - 1;
+                    ok = warp_wait(&bar[kD2Full + (t & 1)], (t >> 1) & 1, err, 0x724) && ok;
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t col = (uint32_t)((t & 1) * 128);
+                    uint32_t v[EC], sv = 0;
+                    if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
+                    else tmem_ld8(tmem + lane_base + col + EC * g, v);
+                    if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
+                    tmem_ld_wait();
+                    if (row < D) {
+                        const float w = row_weight(tab[row]);
+                        float4 *dst = reinterpret_cast<float4 *>(Hst_mut + ((size_t)h * D + row) * DH + EC * g);
+#pragma unroll
+                        for (int u = 0; u < EC / 4; ++u) {
+                            float4 x = hreg[u];
+                            x.x = fmaf(w, __uint_as_float(v[4 * u + 0]), x.x);
+                            x.y = fmaf(w, __uint_as_float(v[4 * u + 1]), x.y);
+                            x.z = fmaf(w, __uint_as_float(v[4 * u + 2]), x.z);
+                            x.w = fmaf(w, __uint_as_float(v[4 * u + 3]), x.w);
+                            dst[u] = x;
+                        }
+                        if (g == 0) s_mut[(size_t)h * D + row] = fmaf(w, __uint_as_float(sv), sreg);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar[kD2Empty + (t & 1)]);
+                }
             }
         }
     }
 
     // teardown: every copy and MMA this CTA issued has completed
-    if (tid == 0) {
-        for (int j = issued > kStages ? issued - kStages : 0; j < issued; ++j)
-            mbar_drain(&bar[kBLoad + j % kStages], (j / kStages) & 1, err, 0x706);
-        mma_commit(&bar[kBDrain]);
-        mbar_drain(&bar[kBDrain], 0, err, 0x707);
+    __syncthreads();
+    if (warp == kProducerWarp && lane == 0)
+        for (int st = issued > NST ? issued - NST : 0; st < issued; ++st)
+            mbar_drain(&bar[kStFull + st % NST], (st / NST) & 1, err, 0x731);
+    if (warp == kMmaWarp && lane == 0) {
+        mma_commit(&bar[kDrain]);
+        mbar_drain(&bar[kDrain], 0, err, 0x732);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -472,9 +611,9 @@ cudaError_t launch(const float *Hst, const float *s, const __nv_bfloat16 *kc,
     cudaError_t e = cudaFuncSetAttribute(sre_tc_kernel<DH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    sre_tc_kernel<DH><<<nh, kST, bytes, stream>>>(Hst, s, kc, vc, (long)cand_stride * DH, pos,
-                                                  cand_stride, n, keep, eps, merge, scores,
-                                                  keep_idx, Hst_mut, s_mut, err);
+    sre_tc_kernel<DH><<<nh, kThreads, bytes, stream>>>(Hst, s, kc, vc, (long)cand_stride * DH,
+                                                       pos, cand_stride, n, keep, eps, merge,
+                                                       scores, keep_idx, Hst_mut, s_mut, err);
     return after_launch();
 }
 
@@ -483,9 +622,10 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 }  // namespace
 
 bool sre_tc_applies(int dtype, int d, int n, const float *Hst, const float *s,
-                    const float *Hst_mut, const float *s_mut) {
+                    const float *Hst_mut, const float *s_mut, const void *kc, const void *vc) {
     return dtype == 1 && (d == 32 || d == 64) && n >= 1 && n <= kNMax && aligned16(Hst) &&
-           aligned16(s) && aligned16(Hst_mut) && aligned16(s_mut);
+           aligned16(s) && aligned16(Hst_mut) && aligned16(s_mut) && aligned16(kc) &&
+           aligned16(vc);
 }
 
 cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void *vc,
