@@ -23,11 +23,12 @@
 // exactly into two bf16 parts), then H[r] += w_r D2[r][0..d-1] and
 // s[r] += w_r D2[r][d] in fp32.
 //
-// One CTA per head (bf16 candidates, d = 32 or 64, at most 256 of them), 18
-// warps: 16 workers (operand conversion and epilogues; warp w reads tensor-
-// memory lanes 32 (w % 4) ..), a producer warp (bulk copies of the state),
-// an MMA warp (one elected lane issues). Roles hand work over through
-// mbarrier rings; every wait is bounded.
+// One CTA per head (bf16 candidates, d = 32 or 64, at most 256 of them), 32
+// warps in four roles that hand work over through mbarrier rings (every wait
+// bounded): 16 epilogue warps (warp w reads tensor-memory lanes 32 (w % 4) ..
+// and a quarter of the columns), 14 builder warps (operand conversion), a
+// producer warp (bulk copies of the state) and an MMA warp (one lane issues).
+// Conversion, MMAs and epilogues of consecutive indices overlap.
 #include "kata_common.cuh"
 #include "kata_internal.h"
 #include "sm100.cuh"
@@ -39,15 +40,17 @@ namespace {
 using namespace sm100;
 using tc::warp_wait;
 
-constexpr int kWorkers = 512;           // 16 worker warps
-constexpr int kThreads = kWorkers + 64;  // + producer warp + MMA warp
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
+constexpr int kEpiWarps = 16;           // epilogue warps: TMEM lane quadrant x column group
+constexpr int kBuildWarps = 14;         // operand builder warps
+constexpr int kEpi = kEpiWarps * 32;
+constexpr int kBuild = kBuildWarps * 32;
+constexpr int kProducerWarp = kEpiWarps + kBuildWarps;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kLR = 64;                 // packed rows per staging copy
 constexpr int kNMax = 256;              // candidates per head
 constexpr int kMR = 128;                // packed rows per merge tile
 constexpr int kMK = 32;                 // merged candidates per merge K chunk
-constexpr int kLag = 2;                 // the epilogue of a trails the build of a by this
 constexpr int kNB = 3;                  // U_a operand buffers
 constexpr int kND = 3;                  // D_a accumulators in tensor memory
 constexpr int kNA = 4;                  // merge operand buffers
@@ -93,6 +96,13 @@ __device__ __forceinline__ float row_weight(uint16_t ab) {
     return (ab >> 8) != (ab & 255) ? kSqrt2f : 1.f;
 }
 
+// Hint: bring [p, p + bytes) into L2 (16-byte aligned, a multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // 32 lanes x 8 or 1 consecutive 32-bit tensor-memory columns.
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -106,15 +116,15 @@ __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t &r) {
 
 enum SreBar {
     kStFull = 0,                     // kStSlots: a staging copy landed (tx count)
-    kStEmpty = kStFull + kStSlots,   // kStSlots: every worker warp is done with a copy
-    kBbFull = kStEmpty + kStSlots,   // kNB: U_a written (worker warps)
+    kStEmpty = kStFull + kStSlots,   // kStSlots: every builder warp is done with a copy
+    kBbFull = kStEmpty + kStSlots,   // kNB: U_a written (builder warps)
     kBbEmpty = kBbFull + kNB, // kNB: the MMAs reading U_a completed
     kDFull = kBbEmpty + kNB,  // kND: D_a complete
-    kDEmpty = kDFull + kND,   // kND: D_a read (worker warps)
-    kA2Full = kDEmpty + kND,  // kNA: a merge operand chunk written
+    kDEmpty = kDFull + kND,   // kND: D_a read (epilogue warps)
+    kA2Full = kDEmpty + kND,  // kNA: a merge operand chunk written (builder warps)
     kA2Empty = kA2Full + kNA, // kNA: the MMAs reading it completed
     kD2Full = kA2Empty + kNA, // 2: a merge tile's D2 complete
-    kD2Empty = kD2Full + 2,   // 2: D2 read (worker warps)
+    kD2Empty = kD2Full + 2,   // 2: D2 read (epilogue warps)
     kDrain = kD2Empty + 2,    // teardown: every MMA completed
     kBarCount = kDrain + 1
 };
@@ -127,7 +137,7 @@ struct SreCfg {
     static constexpr int NCH = DH / 8;          // 16-byte chunks per row
     static constexpr int N1 = DH + 16;          // score MMA N: [H | s | 0] columns
     static constexpr int N2 = DH + 16;          // merge MMA N: [v | 1 | 0]
-    static constexpr int EC = DH / 4;           // epilogue columns per worker warp
+    static constexpr int EC = DH / 4;           // epilogue columns per epilogue warp
     static constexpr int NST = DH == 64 ? 6 : 10;
     static constexpr int NL = (D + kLR - 1) / kLR;  // staging copies
     static constexpr int STG = ((kLR * DH + kLR) * 4 + 1023) / 1024 * 1024;
@@ -162,6 +172,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
     using L = SreCfg<DH>;
     constexpr int D = L::D, RB = L::RB, N1 = L::N1, N2 = L::N2, EC = L::EC, NST = L::NST;
     constexpr int NL = L::NL;
+    constexpr int NT2 = (D + kMR - 1) / kMR;  // merge tiles
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -183,31 +194,33 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
     const float *sh = s + (size_t)h * D;
     const __nv_bfloat16 *kh = kc + (size_t)h * cand_head_stride;
     const __nv_bfloat16 *vh = vc + (size_t)h * cand_head_stride;
-    const bool worker = warp < kProducerWarp;
-    const int qd = warp & 3, g = (warp >> 2) & 3;  // worker: lane quadrant, column group
+    const bool epi = warp < kEpiWarps;
+    const bool builder = warp >= kEpiWarps && warp < kEpiWarps + kBuildWarps;
+    const int btid = tid - kEpi;                   // builder thread index
+    const int qd = warp & 3, g = (warp >> 2) & 3;  // epilogue: lane quadrant, column group
     const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
 
     // ---------------- set-up ----------------
     if (tid == 0) {
         for (int i = 0; i < NST; ++i) {
             mbar_init(&bar[kStFull + i], 1);
-            mbar_init(&bar[kStEmpty + i], 16);
+            mbar_init(&bar[kStEmpty + i], kBuildWarps);
         }
         for (int i = 0; i < kNB; ++i) {
-            mbar_init(&bar[kBbFull + i], 16);
+            mbar_init(&bar[kBbFull + i], kBuildWarps);
             mbar_init(&bar[kBbEmpty + i], 1);
         }
         for (int i = 0; i < kND; ++i) {
             mbar_init(&bar[kDFull + i], 1);
-            mbar_init(&bar[kDEmpty + i], 16);
+            mbar_init(&bar[kDEmpty + i], kEpiWarps);
         }
         for (int i = 0; i < kNA; ++i) {
-            mbar_init(&bar[kA2Full + i], 16);
+            mbar_init(&bar[kA2Full + i], kBuildWarps);
             mbar_init(&bar[kA2Empty + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar[kD2Full + i], 1);
-            mbar_init(&bar[kD2Empty + i], 16);
+            mbar_init(&bar[kD2Empty + i], kEpiWarps);
         }
         mbar_init(&bar[kDrain], 1);
         cta_abort_clear();
@@ -218,9 +231,10 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
         tmem_relinquish();
     }
     build_pair_table(tab, DH);
-    if (worker) {
+    if (epi || builder) {
+        constexpr int nt = kEpi + kBuild;
         // candidate keys as the score MMA's A operand (zero rows past n)
-        for (int idx = tid; idx < nmt * 128 * L::NCH; idx += kWorkers) {
+        for (int idx = tid; idx < nmt * 128 * L::NCH; idx += nt) {
             const int c = idx / L::NCH, ch = idx % L::NCH;
             uint4 x = make_uint4(0, 0, 0, 0);
             if (c < n) x = *reinterpret_cast<const uint4 *>(kh + (size_t)c * DH + ch * 8);
@@ -228,7 +242,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
         }
         // rows DH + 1 .. N1 - 1 of every U_a buffer and part stay zero
         constexpr int zrows = N1 - DH - 1;
-        for (int idx = tid; idx < kNB * 2 * zrows * L::NCH; idx += kWorkers) {
+        for (int idx = tid; idx < kNB * 2 * zrows * L::NCH; idx += nt) {
             const int part = idx / (zrows * L::NCH), rem = idx % (zrows * L::NCH);
             const int row = DH + 1 + rem / L::NCH, ch = rem % L::NCH;
             *reinterpret_cast<uint4 *>(sm + L::OFF_BB + part * L::BPART + kmaj_off<RB>(row, ch)) =
@@ -269,6 +283,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
         }
     } else if (warp == kMmaWarp) {
         const uint32_t id1 = idesc_bf16(128, N1, 0, 0);
+        const uint32_t ka0 = smem_u32(KA);
         for (int a = 0; a < DH; ++a) {
             const int i = a % kNB, j = a % kND;
             ok = warp_wait(&bar[kBbFull + i], (a / kNB) & 1, err, 0x712) && ok;
@@ -280,7 +295,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                 const int ks0 = a / 16;
                 for (int mt = 0; mt < nmt; ++mt) {
                     const uint32_t d = tmem + (uint32_t)((j * nmt + mt) * N1);
-                    const uint32_t ka = smem_u32(KA + mt * 128 * RB);
+                    const uint32_t ka = ka0 + (uint32_t)(mt * 128 * RB);
                     for (int ks = ks0; ks < L::KS; ++ks) {
                         mma_ss(d, kmaj_desc_rb<RB>(ka, ks), kmaj_desc_rb<RB>(bh, ks), id1,
                                ks > ks0 ? 1u : 0u);
@@ -292,32 +307,42 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
             }
             __syncwarp();
         }
-    } else {
+    } else if (builder) {
         int waited = 0, released = 0;  // staging copies waited for / released (warp-uniform)
-        uint4 kreg[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        for (int it = 0; it < DH + kLag && ok; ++it) {
-            if (it < DH) {  // U_it: rows m (value columns and the normaliser), K = b
-                const int a = it, i = a % kNB;
-                const int first = packed_row_base(a, DH), last = first + DH - 1 - a;
-                while (waited <= last / kLR && ok) {
-                    ok = warp_wait(&bar[kStFull + waited % NST], (waited / NST) & 1, err, 0x714) && ok;
-                    ++waited;
-                }
-                if (a >= kNB) ok = warp_wait(&bar[kBbEmpty + i], ((a / kNB) - 1) & 1, err, 0x715) && ok;
-                if (!ok) break;
-                uint8_t *Bh = sm + L::OFF_BB + i * 2 * L::BPART, *Bl = Bh + L::BPART;
-                const int ch0 = (a / 16) * 2, ntask = (DH + 1) * (L::NCH - ch0);
-                for (int idx = tid; idx < ntask; idx += kWorkers) {
-                    const int m = idx % (DH + 1), ch = ch0 + idx / (DH + 1);
-                    // rows of b = 8 ch .. 8 ch + 7 (those with b < a are zero):
-                    // consecutive packed rows, in at most two staging copies
-                    const int b0 = ch * 8, rs = first + (b0 > a ? b0 - a : 0);
-                    const int st0 = rs / kLR;
-                    const float *p0 = reinterpret_cast<const float *>(sm + L::OFF_STG + (st0 % NST) * L::STG);
+        for (int a = 0; a < DH && ok; ++a) {  // U_a: rows m (value columns, the normaliser), K = b
+            const int i = a % kNB;
+            const int first = packed_row_base(a, DH), last = first + DH - 1 - a;
+            while (waited <= last / kLR && ok) {
+                ok = warp_wait(&bar[kStFull + waited % NST], (waited / NST) & 1, err, 0x714) && ok;
+                ++waited;
+            }
+            if (a >= kNB) ok = warp_wait(&bar[kBbEmpty + i], ((a / kNB) - 1) & 1, err, 0x715) && ok;
+            if (!ok) break;
+            uint8_t *Bh = sm + L::OFF_BB + i * 2 * L::BPART, *Bl = Bh + L::BPART;
+            const int ch0 = (a / 16) * 2, ntask = (DH + 1) * (L::NCH - ch0);
+            for (int idx = btid; idx < ntask; idx += kBuild) {
+                const int m = idx % (DH + 1), ch = ch0 + idx / (DH + 1);
+                // rows of b = 8 ch .. 8 ch + 7 (those with b < a are zero):
+                // consecutive packed rows, in at most two staging copies
+                const int b0 = ch * 8, rs = first + (b0 > a ? b0 - a : 0);
+                const int st0 = rs / kLR, lr0 = rs - st0 * kLR;
+                const float *p0 = reinterpret_cast<const float *>(sm + L::OFF_STG + (st0 % NST) * L::STG);
+                float x[8];
+                if (b0 > a && lr0 + 7 < kLR) {
+                    // common case: eight rows of one staging copy, all off the diagonal
+                    if (m < DH) {
+                        const float *pp = p0 + lr0 * DH + m;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) x[u] = kSqrt2f * pp[u * DH];
+                    } else {
+                        const float *pp = p0 + kLR * DH + lr0;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) x[u] = kSqrt2f * pp[u];
+                    }
+                } else {
                     const float *p1 = reinterpret_cast<const float *>(sm + L::OFF_STG + ((st0 + 1) % NST) * L::STG);
                     const int col = m < DH ? m : kLR * DH;  // value column, or the normaliser
                     const int rstride = m < DH ? DH : 1;
-                    float x[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int b = b0 + u, bb = b > a ? b : a;  // rows b < a are not read
@@ -326,63 +351,61 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                         const float val = pp[col];
                         x[u] = b > a ? kSqrt2f * val : (b == a ? val : 0.f);
                     }
-                    uint4 hi, lo;
-                    split8(x, hi, lo);
-                    *reinterpret_cast<uint4 *>(Bh + kmaj_off<RB>(m, ch)) = hi;
-                    *reinterpret_cast<uint4 *>(Bl + kmaj_off<RB>(m, ch)) = lo;
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kBbFull + i]);
-                // staging copies whose rows all come before the next index
-                const int lim = a == DH - 1 ? NL : packed_row_base(a + 1, DH) / kLR;
-                for (; released < lim; ++released)
-                    if (lane == 0) mbar_arrive(&bar[kStEmpty + released % NST]);
+                uint4 hi, lo;
+                split8(x, hi, lo);
+                *reinterpret_cast<uint4 *>(Bh + kmaj_off<RB>(m, ch)) = hi;
+                *reinterpret_cast<uint4 *>(Bl + kmaj_off<RB>(m, ch)) = lo;
             }
-            if (it >= kLag) {  // acc += k_c[a] D_a[c][columns of this warp]
-                const int a = it - kLag, j = a % kND;
-                ok = warp_wait(&bar[kDFull + j], (a / kND) & 1, err, 0x716) && ok;
-                if (!ok) break;
-                tc_fence_after();
-                if ((a & 7) == 0) {  // this thread's candidates' keys a .. a + 7
-                    kreg[0] = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(qd * 32 + lane, a >> 3));
-                    if (nmt > 1)
-                        kreg[1] = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(128 + qd * 32 + lane, a >> 3));
-                }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kBbFull + i]);
+            // staging copies whose rows all come before the next index
+            const int lim = a == DH - 1 ? NL : packed_row_base(a + 1, DH) / kLR;
+            for (; released < lim; ++released)
+                if (lane == 0) mbar_arrive(&bar[kStEmpty + released % NST]);
+        }
+    } else if (epi) {
+        for (int a = 0; a < DH && ok; ++a) {  // acc += k_c[a] D_a[c][columns of this warp]
+            const int j = a % kND;
+            ok = warp_wait(&bar[kDFull + j], (a / kND) & 1, err, 0x716) && ok;
+            if (!ok) break;
+            tc_fence_after();
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    if (mt >= nmt) break;
-                    const uint32_t col = (uint32_t)((j * nmt + mt) * N1);
-                    uint32_t v[EC], sv = 0u;
-                    if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
-                    else tmem_ld8(tmem + lane_base + col + EC * g, v);
-                    if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
-                    tmem_ld_wait();
-                    const uint4 k4 = kreg[mt];
-                    const uint32_t kw = (a & 4) ? ((a & 2) ? k4.w : k4.z) : ((a & 2) ? k4.y : k4.x);
-                    const float kca = (a & 1) ? hi_f32(kw) : lo_f32(kw);
+            for (int mt = 0; mt < 2; ++mt) {
+                if (mt >= nmt) break;
+                if (mt * 128 + qd * 32 >= n) continue;  // no candidate in these lanes
+                const uint32_t col = (uint32_t)((j * nmt + mt) * N1);
+                uint32_t v[EC], sv = 0u;
+                if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
+                else tmem_ld8(tmem + lane_base + col + EC * g, v);
+                if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
+                const int c = mt * 128 + qd * 32 + lane;
+                const uint16_t kb = *reinterpret_cast<const uint16_t *>(
+                    KA + kmaj_off<RB>(c, a >> 3) + (a & 7) * 2);
+                tmem_ld_wait();
+                const float kca = lo_f32(kb);
 #pragma unroll
-                    for (int u = 0; u < EC; ++u)
-                        acc[mt][u] = fmaf(kca, __uint_as_float(v[u]), acc[mt][u]);
-                    sacc[mt] = fmaf(kca, __uint_as_float(sv), sacc[mt]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kDEmpty + j]);
+                for (int u = 0; u < EC; ++u)
+                    acc[mt][u] = fmaf(kca, __uint_as_float(v[u]), acc[mt][u]);
+                sacc[mt] = fmaf(kca, __uint_as_float(sv), sacc[mt]);
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[kDEmpty + j]);
         }
     }
     ok = bar_sync_and(0, kThreads, ok);
 
-    // ---------------- 2. SRE and the kept set (workers) ----------------
+    // ---------------- 2. SRE and the kept set (epilogue warps) ----------------
     const int m_keep = keep < n ? keep : n;
     const int nm = n - m_keep;
-    if (ok && worker) {
+    if (ok && epi) {
         if (g == 0) {
             den[qd * 32 + lane] = sacc[0];
             if (nmt > 1) den[128 + qd * 32 + lane] = sacc[1];
         }
-        bar_sync_and(1, kWorkers, true);
+        bar_sync_and(1, kEpi, true);
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
             const int c = mt * 128 + qd * 32 + lane;
@@ -404,47 +427,68 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                 sqp[g * kNMax + c] = part;
             }
         }
-        bar_sync_and(1, kWorkers, true);
+        bar_sync_and(1, kEpi, true);
         if (tid < n) {
             const float e2 = (sqp[tid] + sqp[kNMax + tid]) + (sqp[2 * kNMax + tid] + sqp[3 * kNMax + tid]);
             sc[tid] = isnan(e2) ? -INFINITY : e2;  // a total order even for 0/0 scores
             cpos[tid] = pos[(size_t)h * pos_head_stride + tid];
             if (scores) scores[(size_t)h * n + tid] = sc[tid];
         }
-        bar_sync_and(1, kWorkers, true);
-        if (tid < n) {
-            const float si = sc[tid];
-            const int pi = cpos[tid];
+        bar_sync_and(1, kEpi, true);
+        {   // rank among all candidates: two threads per candidate, each half of the others
+            const int c = tid >> 1, hf = tid & 1, j0 = hf ? n / 2 : 0, j1 = hf ? n : n / 2;
             int rank = 0;
-            for (int c = 0; c < n; ++c) {
-                const float sj = sc[c];
-                const int pj = cpos[c];
-                rank += sj > si || (sj == si && (pj < pi || (pj == pi && c < tid)));
+            if (c < n) {
+                const float si = sc[c];
+                const int pi = cpos[c];
+#pragma unroll 4
+                for (int jj = j0; jj < j1; ++jj) {
+                    const float sj = sc[jj];
+                    const int pj = cpos[jj];
+                    rank += sj > si || (sj == si && (pj < pi || (pj == pi && jj < c)));
+                }
             }
-            kflag[tid] = rank < m_keep;
-        }
-        bar_sync_and(1, kWorkers, true);
-        if (tid < n) {
-            const int pi = cpos[tid];
-            if (kflag[tid]) {
-                int pr = 0;
-                for (int c = 0; c < n; ++c)
-                    pr += kflag[c] && (cpos[c] < pi || (cpos[c] == pi && c < tid));
-                if (pr < m_keep) keep_idx[(size_t)h * m_keep + pr] = tid;
-            } else {
-                int mr = 0;
-                for (int c = 0; c < tid; ++c) mr += !kflag[c];
-                mlist[mr] = tid;
+            rank += __shfl_xor_sync(0xFFFFFFFFu, rank, 1);
+            if (c < n && hf == 0) kflag[c] = rank < m_keep;
+            bar_sync_and(1, kEpi, true);
+            // kept: rank by position among the kept; merged: rank by slot among the merged
+            int cnt = 0;
+            bool kept = false;
+            if (c < n) {
+                kept = kflag[c] != 0;
+                const int pi = cpos[c];
+#pragma unroll 4
+                for (int jj = j0; jj < j1; ++jj) {
+                    const int kj = kflag[jj];
+                    cnt += kept ? (kj && (cpos[jj] < pi || (cpos[jj] == pi && jj < c)))
+                                : (!kj && jj < c);
+                }
+            }
+            cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
+            if (c < n && hf == 0) {
+                if (kept) {
+                    if (cnt < m_keep) keep_idx[(size_t)h * m_keep + cnt] = c;
+                } else {
+                    mlist[cnt] = c;
+                }
             }
         }
+    }
+    if (ok && merge && nm > 0 && warp == kProducerWarp && lane == 0) {
+        // the merge reads the state again: ask L2 for it while the epilogue warps rank
+        for (int t = 0; t < NT2; ++t) {
+            const int rows = D - t * kMR < kMR ? D - t * kMR : kMR;
+            prefetch_l2(Hh + (size_t)t * kMR * DH, (uint32_t)(rows * DH * 4));
+        }
+        prefetch_l2(sh, (uint32_t)(D * 4));
     }
     __syncthreads();
 
     // ---------------- 3. merge ----------------
     if (ok && merge && nm > 0) {
         const int nk2 = (nm + kMK - 1) / kMK;
-        constexpr int NT2 = (D + kMR - 1) / kMR;
         uint8_t *B2 = sm + L::OFF_B2;
+        uint16_t *kmT = reinterpret_cast<uint16_t *>(sm + L::OFF_KMT);
         if (warp == kMmaWarp) {
             const uint32_t id2 = idesc_bf16(128, N2, 0, 0);
             for (int t = 0; t < NT2 && ok; ++t) {
@@ -472,10 +516,20 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                     __syncwarp();
                 }
             }
-        } else if (worker) {
+        } else if (builder) {
+            // merged keys, transposed: kmT[a][mi] (zero past nm)
+            for (int idx = btid; idx < L::NCH * nk2 * kMK; idx += kBuild) {
+                const int mi = idx % (nk2 * kMK), a8 = idx / (nk2 * kMK);
+                uint4 x = make_uint4(0, 0, 0, 0);
+                if (mi < nm) x = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(mlist[mi], a8));
+                const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    kmT[(a8 * 8 + u) * kKmtPitch + mi] = (uint16_t)(xw[u >> 1] >> ((u & 1) * 16));
+            }
             // B2 (K-major), chunk q: row e < DH is v[e] of merged candidates
             // 32 q .. 32 q + 31, row DH is 1, rows above are 0 (zero past nm)
-            for (int idx = tid; idx < nk2 * N2 * 4; idx += kWorkers) {
+            for (int idx = btid; idx < nk2 * N2 * 4; idx += kBuild) {
                 const int q = idx / (N2 * 4), rem = idx % (N2 * 4);
                 const int kg = rem / N2, e = rem % N2;
                 uint32_t bv[8];
@@ -495,38 +549,18 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                     make_uint4(bv[0] | (bv[1] << 16), bv[2] | (bv[3] << 16),
                                bv[4] | (bv[5] << 16), bv[6] | (bv[7] << 16));
             }
-            // merged keys, transposed: kmT[a][mi] (zero past nm)
-            uint16_t *kmT = reinterpret_cast<uint16_t *>(sm + L::OFF_KMT);
-            for (int idx = tid; idx < L::NCH * nk2 * kMK; idx += kWorkers) {
-                const int mi = idx % (nk2 * kMK), a8 = idx / (nk2 * kMK);
-                uint4 x = make_uint4(0, 0, 0, 0);
-                if (mi < nm) x = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(mlist[mi], a8));
-                const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    kmT[(a8 * 8 + u) * kKmtPitch + mi] = (uint16_t)(xw[u >> 1] >> ((u & 1) * 16));
-            }
-            bar_sync_and(1, kWorkers, true);
-            float4 hreg[EC / 4];
-            float sreg = 0.f;
-            for (int it = 0; it <= NT2 && ok; ++it) {
-                const int row = (it - 1) * kMR + qd * 32 + lane;  // epilogue row (tile it - 1)
-                if (it >= 1 && row < D) {  // read early, used after this iteration's build
-                    const float4 *src = reinterpret_cast<const float4 *>(Hh + (size_t)row * DH + EC * g);
-#pragma unroll
-                    for (int u = 0; u < EC / 4; ++u) hreg[u] = src[u];
-                    if (g == 0) sreg = sh[row];
-                }
-                if (it < NT2) {
-                    for (int q = 0; q < nk2; ++q) {
-                        const int ci = it * nk2 + q, slot = ci % kNA;
-                        if (ci >= kNA)
-                            ok = warp_wait(&bar[kA2Empty + slot], ((ci / kNA) - 1) & 1, err, 0x723) && ok;
-                        if (!ok) break;
-                        uint8_t *Ah = sm + L::OFF_A2 + slot * 2 * L::A2PART, *Al = Ah + L::A2PART;
-                        // tile row rr, merged candidates 32 q + 8 kg .. +7 (kg warp-uniform)
-                        const int rr = tid & 127, kg = tid >> 7;
-                        const int r = it * kMR + rr;
+            bar_sync_and(2, kBuild, true);  // kmT complete
+            for (int t = 0; t < NT2 && ok; ++t) {
+                for (int q = 0; q < nk2; ++q) {
+                    const int ci = t * nk2 + q, slot = ci % kNA;
+                    if (ci >= kNA)
+                        ok = warp_wait(&bar[kA2Empty + slot], ((ci / kNA) - 1) & 1, err, 0x723) && ok;
+                    if (!ok) break;
+                    uint8_t *Ah = sm + L::OFF_A2 + slot * 2 * L::A2PART, *Al = Ah + L::A2PART;
+                    // tile row rr, merged candidates 32 q + 8 kg .. +7
+                    for (int idx = btid; idx < 4 * kMR; idx += kBuild) {
+                        const int rr = idx & (kMR - 1), kg = idx >> 7;
+                        const int r = t * kMR + rr;
                         float x[8];
                         if (r < D) {
                             const int ab = tab[r], col = q * kMK + kg * 8;
@@ -546,40 +580,64 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                         split8(x, hi, lo);
                         *reinterpret_cast<uint4 *>(Ah + kmaj_off<64>(rr, kg)) = hi;
                         *reinterpret_cast<uint4 *>(Al + kmaj_off<64>(rr, kg)) = lo;
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bar[kA2Full + slot]);
                     }
-                    if (!ok) break;
-                }
-                if (it >= 1) {  // H[r] += w_r D2[r], s[r] += w_r D2[r][DH]
-                    const int t = it - 1;
-                    ok = warp_wait(&bar[kD2Full + (t & 1)], (t >> 1) & 1, err, 0x724) && ok;
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t col = (uint32_t)((t & 1) * 128);
-                    uint32_t v[EC], sv = 0;
-                    if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
-                    else tmem_ld8(tmem + lane_base + col + EC * g, v);
-                    if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
-                    tmem_ld_wait();
-                    if (row < D) {
-                        const float w = row_weight(tab[row]);
-                        float4 *dst = reinterpret_cast<float4 *>(Hst_mut + ((size_t)h * D + row) * DH + EC * g);
-#pragma unroll
-                        for (int u = 0; u < EC / 4; ++u) {
-                            float4 x = hreg[u];
-                            x.x = fmaf(w, __uint_as_float(v[4 * u + 0]), x.x);
-                            x.y = fmaf(w, __uint_as_float(v[4 * u + 1]), x.y);
-                            x.z = fmaf(w, __uint_as_float(v[4 * u + 2]), x.z);
-                            x.w = fmaf(w, __uint_as_float(v[4 * u + 3]), x.w);
-                            dst[u] = x;
-                        }
-                        if (g == 0) s_mut[(size_t)h * D + row] = fmaf(w, __uint_as_float(sv), sreg);
-                    }
-                    tc_fence_before();
+                    fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar[kD2Empty + (t & 1)]);
+                    if (lane == 0) mbar_arrive(&bar[kA2Full + slot]);
+                }
+            }
+        } else if (epi) {
+            // the state rows of each tile are read two tiles ahead, into one of two
+            // register sets (the tile's parity picks it)
+            float4 hr0[EC / 4], hr1[EC / 4];
+            float sr0 = 0.f, sr1 = 0.f;
+            auto load_tile = [&](int t, float4 (&hr)[EC / 4], float &sr) {
+                const int row = t * kMR + qd * 32 + lane;
+                if (t < NT2 && row < D) {
+                    const float4 *src = reinterpret_cast<const float4 *>(Hh + (size_t)row * DH + EC * g);
+#pragma unroll
+                    for (int u = 0; u < EC / 4; ++u) hr[u] = src[u];
+                    if (g == 0) sr = sh[row];
+                }
+            };
+            // H[r] += w_r D2[r], s[r] += w_r D2[r][DH] for tile t (its state in hr)
+            auto finish = [&](int t, float4 (&hr)[EC / 4], float &sr) {
+                const int row = t * kMR + qd * 32 + lane;
+                ok = warp_wait(&bar[kD2Full + (t & 1)], (t >> 1) & 1, err, 0x724) && ok;
+                if (!ok) return;
+                tc_fence_after();
+                const uint32_t col = (uint32_t)((t & 1) * 128);
+                uint32_t v[EC], sv = 0;
+                if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
+                else tmem_ld8(tmem + lane_base + col + EC * g, v);
+                if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
+                tmem_ld_wait();
+                if (row < D) {
+                    const float w = row_weight(tab[row]);
+                    float4 *dst = reinterpret_cast<float4 *>(Hst_mut + ((size_t)h * D + row) * DH + EC * g);
+#pragma unroll
+                    for (int u = 0; u < EC / 4; ++u) {
+                        float4 x = hr[u];
+                        x.x = fmaf(w, __uint_as_float(v[4 * u + 0]), x.x);
+                        x.y = fmaf(w, __uint_as_float(v[4 * u + 1]), x.y);
+                        x.z = fmaf(w, __uint_as_float(v[4 * u + 2]), x.z);
+                        x.w = fmaf(w, __uint_as_float(v[4 * u + 3]), x.w);
+                        dst[u] = x;
+                    }
+                    if (g == 0) s_mut[(size_t)h * D + row] = fmaf(w, __uint_as_float(sv), sr);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar[kD2Empty + (t & 1)]);
+            };
+            load_tile(0, hr0, sr0);
+            load_tile(1, hr1, sr1);
+            for (int t = 0; t < NT2 && ok; t += 2) {
+                finish(t, hr0, sr0);
+                load_tile(t + 2, hr0, sr0);
+                if (t + 1 < NT2 && ok) {
+                    finish(t + 1, hr1, sr1);
+                    load_tile(t + 3, hr1, sr1);
                 }
             }
         }
