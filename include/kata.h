@@ -63,7 +63,8 @@ typedef enum {
     KATA_ERR_UNSUPPORTED = 2, /* valid but not built: d, chunk or dtype */
     KATA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     KATA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out */
-    KATA_ERR_WORKSPACE = 5    /* workspace missing or too small */
+    KATA_ERR_WORKSPACE = 5,   /* workspace missing or too small */
+    KATA_ERR_BOUNDS = 6       /* debug library only: a device-side bounds check failed */
 } kata_status;
 
 typedef enum { KATA_F32 = 0, KATA_BF16 = 1 } kata_dtype; /* dtype of q, k, v */
@@ -136,6 +137,28 @@ KATA_API int kata_prefill_path(int B, int H, int T, int d, int chunk, int dtype)
 KATA_API int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B, int H,
                                       int T, int d, float eps, float *o, unsigned int polls,
                                       void *stream);
+
+/*
+ * The debug library (libkata_debug.so, the same sources built with
+ * -DKATA_DEBUG; no counterpart on the pages) adds device-side bounds checks
+ * where an index comes from device data or a size another kernel produced:
+ * candidate slots, kept and merged lists, cache rows, output rows. A check
+ * that fails records its site code (0xB000 .. 0xBFFF) in the device error
+ * word and the access is skipped, so a bad index turns into a status instead
+ * of a memory fault: the next kata_sync_status() returns KATA_ERR_BOUNDS with
+ * the code in kata_last_error(), and the outputs of that call are invalid.
+ * kata_debug_build() returns 1 in the debug library and 0 in libkata.so.
+ */
+KATA_API int kata_debug_build(void);
+
+/*
+ * Test hook of the debug library: launches one tiny kernel whose checked store
+ * targets index 7 of a 4-element device array, so the check fails, records
+ * site code 0xB001 and skips the store. The next kata_sync_status() returns
+ * KATA_ERR_BOUNDS. The normal library returns KATA_ERR_UNSUPPORTED and
+ * launches nothing (its checks are compiled out).
+ */
+KATA_API int kata_test_bounds_check(void *stream);
 
 /* The two exact forms of a prefill. */
 enum { KATA_FORM_AUTO = 0, KATA_FORM_CHUNKED = 1, KATA_FORM_QUADRATIC = 2 };

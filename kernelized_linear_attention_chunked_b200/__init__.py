@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     SIGNATURES,
     KataError,
+    debug_build,
     decode_step,
     decode_step_feature,
     feature_dim,
@@ -33,5 +34,6 @@ from ._binding import (  # noqa: F401
     sre_score_topk,
     state_prefix,
     sync_status,
+    test_bounds_check,
     test_forced_timeout,
 )

@@ -8,12 +8,15 @@ library is missing, every call raises.
 from __future__ import annotations
 
 import ctypes as C
+import os
 from pathlib import Path
 
 import torch
 
 _PKG = Path(__file__).resolve().parent
-LIB_PATH = _PKG / "libkata.so"
+# KATA_DEBUG=1 in the environment loads the debug library (device-side bounds
+# checks, include/kata.h kata_debug_build) instead of libkata.so.
+LIB_PATH = _PKG / ("libkata_debug.so" if os.environ.get("KATA_DEBUG") == "1" else "libkata.so")
 
 KATA_F32, KATA_BF16 = 0, 1
 _DTYPE = {torch.float32: KATA_F32, torch.bfloat16: KATA_BF16}
@@ -33,6 +36,8 @@ SIGNATURES = {
                           _vp, _sz, _vp]),
     "kata_prefill_path": (_i, [_i, _i, _i, _i, _i, _i]),
     "kata_test_forced_timeout": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _f, _vp, C.c_uint, _vp]),
+    "kata_debug_build": (_i, []),
+    "kata_test_bounds_check": (_i, [_vp]),
     "kata_prefill_ex": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp,
                              _vp, _sz, _vp, _i]),
     "kata_quadratic_max_tokens": (_i, [_i]),
@@ -180,6 +185,17 @@ def test_forced_timeout(q, k, v, polls: int, eps: float = 1e-6, o=None, stream=N
     _check("kata_test_forced_timeout", lib().kata_test_forced_timeout(
         _ptr(q), _ptr(k), _ptr(v), B, Hh, T, d, eps, _ptr(o), polls, _stream(stream)))
     return o
+
+
+def debug_build() -> bool:
+    """True when the loaded library is libkata_debug.so (device-side bounds checks)."""
+    return bool(lib().kata_debug_build())
+
+
+def test_bounds_check(stream=None) -> None:
+    """kata_test_bounds_check: one checked store past the end of a small device
+    array (debug library only); the next sync_status() raises KATA_ERR_BOUNDS."""
+    _check("kata_test_bounds_check", lib().kata_test_bounds_check(_stream(stream)))
 
 
 def prefill_auto_form(B, H, T, d, chunk, dtype, with_state: bool = False) -> str:

@@ -135,6 +135,7 @@ const char *kata_status_string(int status) {
         case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
         case KATA_ERR_TIMEOUT: return "KATA_ERR_TIMEOUT";
         case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
+        case KATA_ERR_BOUNDS: return "KATA_ERR_BOUNDS";
         default: return "KATA_ERR_UNKNOWN";
     }
 }
@@ -155,6 +156,8 @@ int kata_sync_status(void *stream) {
         unsigned int zero = 0;
         e = cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+        if (h >= kata::kErrBoundsFirst && h <= kata::kErrBoundsLast)
+            return fail(KATA_ERR_BOUNDS, "a device-side bounds check failed (site 0x%X)", h);
         return fail(KATA_ERR_TIMEOUT, "a kernel's bounded wait ran out (code 0x%X)", h);
     }
     return KATA_OK;
@@ -434,6 +437,39 @@ int kata_test_forced_timeout(const void *q, const void *k, const void *v, int B,
     cudaError_t e = kata::quad_tc(a, static_cast<cudaStream_t>(stream), polls);
     if (e != cudaSuccess) return cuda_fail(e, "kata_test_forced_timeout launch");
     return KATA_OK;
+}
+
+#ifdef KATA_DEBUG
+namespace {
+__device__ int g_bounds_probe[4];
+// One checked store past the end of a 4-element array: the check records
+// 0xB001 and the store is skipped.
+__global__ void bounds_probe_kernel(int idx) {
+    if (threadIdx.x == 0 && KATA_CHECK(idx >= 0 && idx < 4, 0xB001u)) g_bounds_probe[idx] = 1;
+}
+}  // namespace
+#endif
+
+int kata_debug_build(void) {
+#ifdef KATA_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int kata_test_bounds_check(void *stream) {
+    g_last_error[0] = 0;
+#ifdef KATA_DEBUG
+    KATA_DEBUG_BIND();
+    bounds_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(7);
+    const cudaError_t e = kata::after_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "kata_test_bounds_check launch");
+    return KATA_OK;
+#else
+    (void)stream;
+    return fail(KATA_ERR_UNSUPPORTED, "bounds checks are compiled into libkata_debug.so only");
+#endif
 }
 
 size_t kata_prefill_host_workspace_bytes(int B, int H, int T, int d, int chunk, int dtype) {

@@ -97,7 +97,35 @@ __device__ __forceinline__ float factor_kernel(const float *q, const float *k, i
     return sum;
 }
 
-// Device-side error codes written to the per-device error word.
-enum : unsigned int { kErrNone = 0, kErrTimeout = 1 };
+// Device-side error codes written to the per-device error word. Codes
+// kErrBoundsFirst .. kErrBoundsLast are bounds-check sites of the debug build.
+enum : unsigned int { kErrNone = 0, kErrTimeout = 1, kErrBoundsFirst = 0xB000, kErrBoundsLast = 0xBFFF };
 
 }  // namespace kata
+
+// ------------------------------------------------------------ debug build --
+// Bounds checks of the debug library (compiled with -DKATA_DEBUG): a check
+// that fails records its site code (0xB000 and up) in the device error word,
+// which kata_sync_status reports as KATA_ERR_BOUNDS, and the caller skips the
+// access instead of faulting. In the normal library KATA_CHECK is the
+// constant true and costs nothing. Each translation unit holds its own copy of
+// the pointer to the word; KATA_DEBUG_BIND() (in its launchers, after
+// kata_internal.h) points it at this device's word.
+#ifdef KATA_DEBUG
+static __constant__ unsigned int *kata_dbg_word;
+__device__ __forceinline__ bool kata_dbg_check(bool ok, unsigned int code) {
+    if (!ok && kata_dbg_word) atomicCAS(kata_dbg_word, 0u, code);
+    return ok;
+}
+#define KATA_CHECK(cond, code) kata_dbg_check((cond), (code))
+#define KATA_DEBUG_BIND()                                                     \
+    do {                                                                      \
+        unsigned int *kata_dbg_p = ::kata::device_error_word();               \
+        cudaMemcpyToSymbol(kata_dbg_word, &kata_dbg_p, sizeof(kata_dbg_p));   \
+    } while (0)
+#else
+#define KATA_CHECK(cond, code) true
+#define KATA_DEBUG_BIND() \
+    do {                  \
+    } while (0)
+#endif

@@ -359,8 +359,10 @@ merge_kernel(const float *Hsrc, const float *ssrc, float *Hdst, float *sdst,
             float kx = 0.f, vx = 0.f;
             if (ii < nb) {
                 const int j = mlist[(size_t)h * n + mc + ii];
-                kx = to_f32(kh[(size_t)j * DH + a]);
-                vx = to_f32(vh[(size_t)j * DH + a]);
+                if (KATA_CHECK(j >= 0 && j < n, 0xB304u)) {
+                    kx = to_f32(kh[(size_t)j * DH + a]);
+                    vx = to_f32(vh[(size_t)j * DH + a]);
+                }
             }
             Ks[ii][a] = kx;
             Vs[ii][a] = vx;
@@ -507,6 +509,7 @@ __global__ void lola_append_kernel(const Tin *__restrict__ k, const Tin *__restr
     const int h = blockIdx.x;
     for (int idx = threadIdx.x; idx < U * d; idx += blockDim.x) {
         const int u = idx / d, a = idx % d;
+        if (!KATA_CHECK(nc + u < cap, 0xB301u) || !KATA_CHECK(pstart + u < T, 0xB302u)) continue;
         const size_t src = ((size_t)h * T + pstart + u) * d + a;
         const size_t dst = ((size_t)h * cap + nc + u) * d + a;
         cand_k[dst] = k[src];
@@ -525,6 +528,7 @@ __global__ void lola_compact_kernel(const Tin *__restrict__ src_k, const Tin *__
     for (int idx = threadIdx.x; idx < m * d; idx += blockDim.x) {
         const int rr = idx / d, a = idx % d;
         const int j = keep_idx[(size_t)h * m + rr];
+        if (!KATA_CHECK(j >= 0 && j < cap, 0xB303u)) continue;
         dst_k[((size_t)h * cap + rr) * d + a] = src_k[((size_t)h * cap + j) * d + a];
         dst_v[((size_t)h * cap + rr) * d + a] = src_v[((size_t)h * cap + j) * d + a];
         if (a == 0) dst_pos[(size_t)h * cap + rr] = src_pos[(size_t)h * cap + j];
@@ -722,6 +726,7 @@ cudaError_t sre_score_topk(const float *Hst, const float *s, const void *kc, con
                            int cand_stride, int keep, float eps, int merge, float *scores,
                            int *keep_idx, float *Hst_mut, float *s_mut, void *ws,
                            size_t ws_bytes, cudaStream_t stream) {
+    KATA_DEBUG_BIND();
     (void)ws_bytes;
     const int nh = B * H;
     if (sre_tc_applies(dtype, d, n_cand, Hst, s, Hst_mut, s_mut, kc, vc))
@@ -742,6 +747,7 @@ cudaError_t hybrid_readout(const void *q, const void *k, const void *v, int dtyp
                            const void *cv, int nc, int cap, const float *Hst, const float *s,
                            float eps, float tau, float *o, void *ws, size_t ws_bytes,
                            cudaStream_t stream) {
+    KATA_DEBUG_BIND();
     (void)ws_bytes;
     const int nh = B * H;
     if (dtype == 0)
@@ -761,6 +767,7 @@ cudaError_t lola_run(const void *q, const void *k, const void *v, int dtype, int
                      int T, int d, int window, int cache, float eps, float tau, float *o,
                      float *Hst, float *s, int *kept_pos, void *ws, size_t ws_bytes,
                      cudaStream_t stream) {
+    KATA_DEBUG_BIND();
     (void)ws_bytes;
     const int nh = B * H;
     if (dtype == 0)

@@ -465,9 +465,11 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             int before = 0;
             for (int i = 0; i < j; ++i) before += kflag[i];
             if (kflag[j]) {
-                klist[before] = j;
-                cnext[before] = cand_pos[j];  // candidates are in ascending position
-            } else {
+                if (KATA_CHECK(before < keep, 0xB501u)) {
+                    klist[before] = j;
+                    cnext[before] = cand_pos[j];  // candidates are in ascending position
+                }
+            } else if (KATA_CHECK(j - before < ncand - keep, 0xB502u)) {
                 mlist[j - before] = j;
             }
         }
@@ -704,6 +706,7 @@ size_t lola_fused_scratch_bytes(int nh, int d) {
 cudaError_t lola_fused(const void *q, const void *k, const void *v, int dtype, int nh, int T,
                        int d, int window, int cache, float eps, float tau, float *o, float *Hst,
                        float *s, int *kept_pos, void *scratch, int ncl, cudaStream_t stream) {
+    KATA_DEBUG_BIND();
     float *sc = static_cast<float *>(scratch);
     if (dtype == 0)
         return fused_dispatch<float>(q, k, v, nh, T, d, window, cache, eps, tau, o, Hst, s,

@@ -142,7 +142,7 @@ prefill_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             }
             __syncthreads();
         }
-        if (o && row < cs) {
+        if (o && row < cs && KATA_CHECK(t0 + row < T, 0xB101u)) {
             const float inv = 1.f / (z + eps);
             float *orow = o + xoff + (size_t)(t0 + row) * d + e0 + eq;
             orow[0] = acc0 * inv;
@@ -191,6 +191,7 @@ cudaError_t launch_feature(const PrefillArgs &a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t prefill_simt(const PrefillArgs &a, cudaStream_t stream) {
+    KATA_DEBUG_BIND();
     return a.dtype == 0 ? launch_feature<float>(a, stream)
                         : launch_feature<__nv_bfloat16>(a, stream);
 }

@@ -468,7 +468,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
             if (c < n && hf == 0) {
                 if (kept) {
                     if (cnt < m_keep) keep_idx[(size_t)h * m_keep + cnt] = c;
-                } else {
+                } else if (KATA_CHECK(cnt < nm, 0xB402u)) {
                     mlist[cnt] = c;
                 }
             }
@@ -521,7 +521,8 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
             for (int idx = btid; idx < L::NCH * nk2 * kMK; idx += kBuild) {
                 const int mi = idx % (nk2 * kMK), a8 = idx / (nk2 * kMK);
                 uint4 x = make_uint4(0, 0, 0, 0);
-                if (mi < nm) x = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(mlist[mi], a8));
+                if (mi < nm && KATA_CHECK(mlist[mi] >= 0 && mlist[mi] < n, 0xB401u))
+                    x = *reinterpret_cast<const uint4 *>(KA + kmaj_off<RB>(mlist[mi], a8));
                 const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
@@ -537,7 +538,7 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                 for (int u = 0; u < 8; ++u) {
                     const int mi = q * kMK + kg * 8 + u;
                     uint32_t val = 0;
-                    if (mi < nm) {
+                    if (mi < nm && KATA_CHECK(mlist[mi] >= 0 && mlist[mi] < n, 0xB403u)) {
                         if (e < DH)
                             val = reinterpret_cast<const uint16_t *>(vh)[(size_t)mlist[mi] * DH + e];
                         else if (e == DH)
@@ -692,6 +693,7 @@ cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void 
                    unsigned int *err, cudaStream_t stream) {
     using bf = __nv_bfloat16;
     const bf *k = static_cast<const bf *>(kc), *v = static_cast<const bf *>(vc);
+    KATA_DEBUG_BIND();
     cudaError_t e;
     if (d == 64)
         e = launch<64>(Hst, s, k, v, pos, nh, n, cand_stride, keep, eps, merge, scores, keep_idx,

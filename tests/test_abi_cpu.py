@@ -21,7 +21,7 @@ def header_functions():
 
 def test_header_symbols_exported_and_bound():
     names = header_functions()
-    assert len(names) == 30
+    assert len(names) == 32
     L = kata.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -42,6 +42,7 @@ def test_status_strings_and_helpers():
     assert L.kata_version() >= 100
     assert L.kata_status_string(0) == b"KATA_OK"
     assert L.kata_status_string(4) == b"KATA_ERR_TIMEOUT"
+    assert L.kata_status_string(6) == b"KATA_ERR_BOUNDS"
     assert L.kata_status_string(99) == b"KATA_ERR_UNKNOWN"
     assert kata.launch_count() == 0  # validation failures launch nothing
     for d in (16, 32, 64):
@@ -197,3 +198,37 @@ def test_feature_dims_and_validation():
     assert L.kata_decode_step_feature(FAKE, FAKE, FAKE, 1, 1, 1, 32, 1e-6, 2, 3, FAKE, FAKE,
                                       FAKE, None) == 2
     assert kata.launch_count() == 0
+
+
+def test_bounds_hook_compiled_out_of_the_normal_library():
+    L = kata.lib()
+    if kata.debug_build():
+        pytest.skip("this process loaded the debug library")
+    assert L.kata_debug_build() == 0
+    assert L.kata_test_bounds_check(None) == 2  # KATA_ERR_UNSUPPORTED, nothing launched
+    assert kata.launch_count() == 0
+
+
+def test_debug_library_loads_and_exports_every_symbol():
+    # a separate process: each library carries its own static CUDA runtime
+    import os
+    import subprocess
+    import sys
+    lib_debug = ROOT / "kernelized_linear_attention_chunked_b200" / "libkata_debug.so"
+    if not lib_debug.exists():
+        pytest.skip("libkata_debug.so not built")
+    code = (
+        "import re, sys; sys.path.insert(0, %r)\n"
+        "import kernelized_linear_attention_chunked_b200 as kata\n"
+        "from kernelized_linear_attention_chunked_b200 import _binding\n"
+        "assert _binding.LIB_PATH.name == 'libkata_debug.so'\n"
+        "assert kata.debug_build()\n"
+        "names = re.findall(r'KATA_API\\s+[\\w\\s\\*]+?\\b(\\w+)\\s*\\(', open(%r).read())\n"
+        "L = kata.lib()\n"
+        "assert all(hasattr(L, n) for n in names)\n"
+        "print('ok', len(names))\n" % (str(ROOT), str(HEADER)))
+    env = dict(os.environ, KATA_DEBUG="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == "ok 32"
