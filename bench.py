@@ -171,6 +171,18 @@ def traffic_source(kernel: str, workload: str) -> str:
             f"{rec.get('case', workload)}, kernel source sha {rec['sha']}")
 
 
+def attach_traffic(roof: dict, kernels: list[str], workload: str) -> dict:
+    """Add the recorded ncu DRAM bytes per call (the sum over the call's
+    kernels, one launch each) to a roofline object, or None when any record is
+    missing or stale."""
+    recs = {k: traffic_record(k, workload) for k in kernels}
+    roof["traffic"] = sum(recs.values()) if all(v is not None for v in recs.values()) else None
+    roof["traffic_source"] = "; ".join(f"{k}: {traffic_source(k, workload)}" for k in kernels)
+    if len(kernels) > 1:
+        roof["traffic_per_kernel"] = recs
+    return roof
+
+
 def roofline(seconds: float, flops: float | None, nbytes: float | None, peaks,
              tensor_key: str = "bf16_tflops") -> dict:
     """Roofline of one launch or call that does `flops` algorithmic flops and
@@ -579,7 +591,8 @@ def bench_decode(kata, args, dev, stream, peaks, dist_on, world):
     flops = float(w.B * w.H * 4 * D * (w.d + 1))
     return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B, nsteps, ms),
             "us_per_step": 1e3 * ms_step, "steps": nsteps,
-            "roofline": roofline(ms_step / 1e3, flops, decode_bytes(w), peaks),
+            "roofline": attach_traffic(roofline(ms_step / 1e3, flops, decode_bytes(w), peaks),
+                                       ["decode_kernel"], w.name),
             "bytes_per_step": decode_bytes(w),
             "gpu_launches": launches, "l2": "state 554 MB > 126 MB L2"}
 
@@ -615,9 +628,11 @@ def bench_sre_stress(kata, args, dev, stream, peaks, dist_on, world):
     # fp32 work: phi(k)^T [H | s] for every candidate, then a rank-one update
     # of [H | s] for every merged one (2 flops per multiply-add)
     flops = float(B * H * (n + (n - keep)) * D * (d + 1) * 2)
-    roof = roofline(ms / 1e3, None, nbytes, peaks)
-    roof["note"] = ("HBM roofline of the algorithmic bytes; the scores are fp32 "
-                    "(fp32_tflops gives the arithmetic rate, not a roofline)")
+    roof = attach_traffic(roofline(ms / 1e3, None, nbytes, peaks), ["sre_tc_kernel"],
+                          "sre_b64_h16_d64_n192_keep128")
+    roof["note"] = ("HBM roofline of the algorithmic bytes; the scores run on the tensor "
+                    "cores with split bf16 operands at fp32-level accuracy (fp32_tflops is "
+                    "the method's fp32 operation count per second, not a roofline)")
     return {"workload": "sre_b64_h16_d64_n192_keep128", "ms_per_pass": ms,
             "roofline": roof, "bytes_per_pass": nbytes,
             "fp32_tflops": flops / (ms / 1e3) / 1e12, "flops_per_pass": flops,
@@ -644,7 +659,8 @@ def bench_long_prefill(kata, args, dev, stream, peaks, dist_on, world):
     fl = prefill_flops(w)
     return {"workload": w.name, "tokens_per_s": aggregate_rate(world, w.B * w.T, 1, ms), "ms": ms,
             "form": kata.prefill_auto_form(w.B, w.H, w.T, w.d, w.chunk, torch.bfloat16),
-            "roofline": roofline(ms / 1e3, fl, prefill_bytes(w), peaks),
+            "roofline": attach_traffic(roofline(ms / 1e3, fl, prefill_bytes(w), peaks),
+                                       ["state_kernel", "readout_kernel"], w.name),
             "l2": "inputs 335 MB > 126 MB L2"}
 
 
@@ -686,6 +702,8 @@ def bench_lola(kata, args, dev, stream, peaks, dist_on, world):
     roof["model"] = ("state-streaming model: each of the 127 updates of each head reads and "
                      "writes its 540,800-byte fp32 state once; the state fits in L2, so this "
                      "is a yardstick, not the bytes HBM moves")
+    if run == "fused":
+        attach_traffic(roof, ["lola_fused_kernel"], w.name)
     return {"workload": w.name, "tokens_per_s": world * w.B * w.T / (ms / 1e3), "ms": ms,
             "run": run, "updates": updates, "gpu_launches_per_pass": launches, "roofline": roof,
             "segments_run_ms": ms_seg,
