@@ -21,7 +21,9 @@
 // Merge, 128 packed rows at a time: D2[r][e] = sum_m k_m[a_r] k_m[b_r]
 // [v_m | 1][e] with exact products (the product of two bf16 values splits
 // exactly into two bf16 parts), then H[r] += w_r D2[r][0..d-1] and
-// s[r] += w_r D2[r][d] in fp32.
+// s[r] += w_r D2[r][d] in fp32, added by bulk reductions (the bulk-copy
+// engine reads the update from shared memory and adds it in L2). The kernel
+// merges in place; the host copies the state first for an out-of-place call.
 //
 // One CTA per head (bf16 candidates, d = 32 or 64, at most 256 of them), 32
 // warps in four roles that hand work over through mbarrier rings (every wait
@@ -53,7 +55,7 @@ constexpr int kMR = 128;                // packed rows per merge tile
 constexpr int kMK = 32;                 // merged candidates per merge K chunk
 constexpr int kNB = 3;                  // U_a operand buffers
 constexpr int kND = 3;                  // D_a accumulators in tensor memory
-constexpr int kNA = 4;                  // merge operand buffers
+constexpr int kNA = 2;                  // merge operand buffers
 constexpr int kStSlots = 10;            // staging copies in flight, at most
 constexpr int kKmtPitch = 264;          // merged keys, transposed: row pitch (bank spread)
 constexpr float kSqrt2f = 1.41421356237309515f;
@@ -103,6 +105,20 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
                  : "memory");
 }
 
+// dst (global) += src (shared), elementwise fp32, by the bulk-copy engine; the
+// reduction runs in L2. Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(dst)),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most one bulk group of this thread is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // 32 lanes x 8 or 1 consecutive 32-bit tensor-memory columns.
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -148,7 +164,12 @@ struct SreCfg {
     static constexpr int OFF_KA = 0;
     static constexpr int OFF_STG = OFF_KA + KA_BYTES;
     static constexpr int OFF_BB = OFF_STG + NST * STG;  // [kNB][hi, lo]
-    static constexpr int OFF_B2 = OFF_STG;              // merge: over the staging copies
+    // merge: two images of a tile's state update (w_r D2, rows of DH then the
+    // normaliser column), over the key operand and the staging copies, then B2,
+    // the A2 ring and the transposed merged keys
+    static constexpr int DHB = (kMR * DH * 4 + kMR * 4 + 1023) / 1024 * 1024;
+    static constexpr int OFF_DH = OFF_KA;
+    static constexpr int OFF_B2 = OFF_DH + 2 * DHB;
     static constexpr int OFF_A2 = OFF_B2 + (kNMax / kMK) * B2TILE;  // [kNA][hi, lo]
     static constexpr int OFF_KMT = OFF_A2 + kNA * 2 * A2PART;  // merge: keys [DH][kKmtPitch]
     static constexpr int OFF_TAB = OFF_BB + kNB * 2 * BPART;
@@ -588,59 +609,49 @@ sre_tc_kernel(const float *Hst, const float *s, const __nv_bfloat16 *__restrict_
                 }
             }
         } else if (epi) {
-            // the state rows of each tile are read two tiles ahead, into one of two
-            // register sets (the tile's parity picks it)
-            float4 hr0[EC / 4], hr1[EC / 4];
-            float sr0 = 0.f, sr1 = 0.f;
-            auto load_tile = [&](int t, float4 (&hr)[EC / 4], float &sr) {
-                const int row = t * kMR + qd * 32 + lane;
-                if (t < NT2 && row < D) {
-                    const float4 *src = reinterpret_cast<const float4 *>(Hh + (size_t)row * DH + EC * g);
-#pragma unroll
-                    for (int u = 0; u < EC / 4; ++u) hr[u] = src[u];
-                    if (g == 0) sr = sh[row];
-                }
-            };
-            // H[r] += w_r D2[r], s[r] += w_r D2[r][DH] for tile t (its state in hr)
-            auto finish = [&](int t, float4 (&hr)[EC / 4], float &sr) {
-                const int row = t * kMR + qd * 32 + lane;
-                ok = warp_wait(&bar[kD2Full + (t & 1)], (t >> 1) & 1, err, 0x724) && ok;
-                if (!ok) return;
+            // w_r D2[r] of tile t goes to a shared-memory image of the tile's state
+            // rows (row-major, as in HBM; the normaliser column after them); one
+            // thread adds the image to the state with bulk reductions in L2, so
+            // no thread reads the state
+            for (int t = 0; t < NT2; ++t) {
+                const int b = t & 1, rr = qd * 32 + lane, row = t * kMR + rr;
+                float *img = reinterpret_cast<float *>(sm + L::OFF_DH + b * L::DHB);
+                ok = warp_wait(&bar[kD2Full + b], (t >> 1) & 1, err, 0x724) && ok;
                 tc_fence_after();
-                const uint32_t col = (uint32_t)((t & 1) * 128);
                 uint32_t v[EC], sv = 0;
-                if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
-                else tmem_ld8(tmem + lane_base + col + EC * g, v);
-                if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
-                tmem_ld_wait();
-                if (row < D) {
-                    const float w = row_weight(tab[row]);
-                    float4 *dst = reinterpret_cast<float4 *>(Hst_mut + ((size_t)h * D + row) * DH + EC * g);
-#pragma unroll
-                    for (int u = 0; u < EC / 4; ++u) {
-                        float4 x = hr[u];
-                        x.x = fmaf(w, __uint_as_float(v[4 * u + 0]), x.x);
-                        x.y = fmaf(w, __uint_as_float(v[4 * u + 1]), x.y);
-                        x.z = fmaf(w, __uint_as_float(v[4 * u + 2]), x.z);
-                        x.w = fmaf(w, __uint_as_float(v[4 * u + 3]), x.w);
-                        dst[u] = x;
-                    }
-                    if (g == 0) s_mut[(size_t)h * D + row] = fmaf(w, __uint_as_float(sv), sr);
+                if (ok) {
+                    const uint32_t col = (uint32_t)(b * 128);
+                    if constexpr (EC == 16) tmem_ld16(tmem + lane_base + col + EC * g, v);
+                    else tmem_ld8(tmem + lane_base + col + EC * g, v);
+                    if (g == 0) tmem_ld1(tmem + lane_base + col + DH, sv);
+                    tmem_ld_wait();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar[kD2Empty + (t & 1)]);
-            };
-            load_tile(0, hr0, sr0);
-            load_tile(1, hr1, sr1);
-            for (int t = 0; t < NT2 && ok; t += 2) {
-                finish(t, hr0, sr0);
-                load_tile(t + 2, hr0, sr0);
-                if (t + 1 < NT2 && ok) {
-                    finish(t + 1, hr1, sr1);
-                    load_tile(t + 3, hr1, sr1);
+                if (lane == 0 && ok) mbar_arrive(&bar[kD2Empty + b]);
+                // the reduction that read this image two tiles ago is done reading
+                if (tid == 0 && t >= 2) bulk_wait_read_one();
+                ok = bar_sync_and(1, kEpi, ok);
+                if (!ok) break;
+                const float w = row < D ? row_weight(tab[row]) : 0.f;
+                float4 *dst = reinterpret_cast<float4 *>(img + rr * DH + EC * g);
+#pragma unroll
+                for (int u = 0; u < EC / 4; ++u)
+                    dst[u] = make_float4(w * __uint_as_float(v[4 * u + 0]), w * __uint_as_float(v[4 * u + 1]),
+                                         w * __uint_as_float(v[4 * u + 2]), w * __uint_as_float(v[4 * u + 3]));
+                if (g == 0) img[kMR * DH + rr] = w * __uint_as_float(sv);
+                fence_proxy_async_smem();
+                bar_sync_and(1, kEpi, true);
+                if (tid == 0) {
+                    const int rows = D - t * kMR < kMR ? D - t * kMR : kMR;
+                    bulk_reduce_add_f32(Hst_mut + ((size_t)h * D + (size_t)t * kMR) * DH, img,
+                                        (uint32_t)(rows * DH * 4));
+                    bulk_reduce_add_f32(s_mut + (size_t)h * D + (size_t)t * kMR, img + kMR * DH,
+                                        (uint32_t)(rows * 4));
+                    bulk_commit();
                 }
             }
+            if (tid == 0) bulk_wait_all();  // the reductions are complete before the CTA exits
         }
     }
 
@@ -695,6 +706,19 @@ cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void 
     const bf *k = static_cast<const bf *>(kc), *v = static_cast<const bf *>(vc);
     KATA_DEBUG_BIND();
     cudaError_t e;
+    if (merge && (Hst_mut != Hst || s_mut != s)) {
+        // the kernel merges in place: an out-of-place call works on a copy of the
+        // state in the output buffers (scored there: the same values)
+        const size_t D = (size_t)d * (d + 1) / 2;
+        if ((e = cudaMemcpyAsync(Hst_mut, Hst, (size_t)nh * D * d * 4, cudaMemcpyDeviceToDevice,
+                                 stream)) != cudaSuccess)
+            return e;
+        if ((e = cudaMemcpyAsync(s_mut, s, (size_t)nh * D * 4, cudaMemcpyDeviceToDevice,
+                                 stream)) != cudaSuccess)
+            return e;
+        Hst = Hst_mut;
+        s = s_mut;
+    }
     if (d == 64)
         e = launch<64>(Hst, s, k, v, pos, nh, n, cand_stride, keep, eps, merge, scores, keep_idx,
                        Hst_mut, s_mut, err, stream);
@@ -703,14 +727,6 @@ cudaError_t sre_tc(const float *Hst, const float *s, const void *kc, const void 
                        Hst_mut, s_mut, err, stream);
     else
         return cudaErrorInvalidValue;
-    if (e != cudaSuccess) return e;
-    if (merge && keep >= n && (Hst_mut != Hst || s_mut != s)) {  // nothing to merge: copy through
-        const size_t D = (size_t)d * (d + 1) / 2;
-        if ((e = cudaMemcpyAsync(Hst_mut, Hst, (size_t)nh * D * d * 4, cudaMemcpyDeviceToDevice,
-                                 stream)) != cudaSuccess)
-            return e;
-        e = cudaMemcpyAsync(s_mut, s, (size_t)nh * D * 4, cudaMemcpyDeviceToDevice, stream);
-    }
     return e;
 }
 
