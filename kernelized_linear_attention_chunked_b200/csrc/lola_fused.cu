@@ -56,7 +56,8 @@ constexpr int kNKMax = 256;       // softmax keys per segment (window + cache)
 constexpr int kWMax = 64;         // longest segment
 constexpr int kQMax = 16;         // queries per CTA (a segment over at least 4 CTAs)
 constexpr int kNclMin = 6;        // fewest CTAs per head: D / 6 rows fit one pass of kFT threads
-constexpr int kVPT = 4;           // scoring vectors per thread (x 8 columns)
+constexpr int kVPT = 4;           // scoring vectors per thread of the s column
+constexpr int kVPH = 8;           // scoring vectors per thread of the H columns (x 8 columns)
 
 __device__ __forceinline__ float xv(const float *p) { return *p; }
 __device__ __forceinline__ float xv(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
@@ -132,6 +133,8 @@ struct FusedCfg {
     static constexpr size_t BYTES = (size_t)(OFF_INT + NINT) * 4;
     static_assert(OFF_SS % 4 == 0 && RED % 4 == 0 && BUF % 4 == 0, "16-byte alignment");
     static_assert(R <= kFT, "one state row per thread in the merge");
+    static_assert((DH / 16) * ((R + DH / 16 - 1) / (DH / 16)) <= kFT,
+                  "one (row group, column group) tile per thread in the merge");
 };
 
 // Global scratch per head: partial sums [NCL][kNSMax][DH+1], the full
@@ -249,15 +252,18 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
 
         // ---- B: phi(x)^T [H | s] over this CTA's rows, x = queries + new candidates ----
         {
-            const bool hthr = tid < 32 * CG;  // H columns 4cg..4cg+3 and 4(CG+cg)..+3
-            const bool sthr = warp == 8;      // the s column
-            const int vg = hthr ? tid / CG : lane;  // vectors kVPT vg .. kVPT vg + kVPT - 1
+            // H threads: 8 vectors x 8 columns (4cg..4cg+3 and 4(CG+cg)..+3) each,
+            // so one 16-byte read of shared memory feeds 16 multiply-adds
+            const bool hthr = tid < (kNSMax / kVPH) * CG;
+            const bool sthr = warp == 8;      // the s column: 4 vectors per lane
+            const int nvt = hthr ? kVPH : kVPT;     // vectors per thread
+            const int vg = hthr ? tid / CG : lane;  // vectors nvt vg .. nvt vg + nvt - 1
             const int cg = tid % CG;
-            const bool act = (hthr || sthr) && kVPT * vg < nsc;
+            const bool act = (hthr || sthr) && nvt * vg < nsc;
             const int bx = tid & (kNSMax - 1), brs = tid >> 7;  // phi builder: column, row phase
-            float acc[kVPT][8];
+            float acc[kVPH][8];
 #pragma unroll
-            for (int i = 0; i < kVPT; ++i)
+            for (int i = 0; i < kVPH; ++i)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
             for (int c0 = 0; c0 < nrows; c0 += kRC) {
@@ -277,18 +283,19 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                 }
                 __syncthreads();
                 if (act) {
-                    const float *prow = buf + kVPT * vg;
+                    const float *prow = buf + nvt * vg;
                     if (hthr) {
                         const float4 *hrow = reinterpret_cast<const float4 *>(Hs + c0 * DH);
-#pragma unroll 4
+#pragma unroll 2
                         for (int rr = 0; rr < nr; ++rr) {
                             const float4 p4 = *reinterpret_cast<const float4 *>(prow + rr * kNSMax);
-                            const float pv[kVPT] = {p4.x, p4.y, p4.z, p4.w};
+                            const float4 p5 = *reinterpret_cast<const float4 *>(prow + rr * kNSMax + 4);
+                            const float pv[kVPH] = {p4.x, p4.y, p4.z, p4.w, p5.x, p5.y, p5.z, p5.w};
                             const float4 h0 = hrow[rr * (DH / 4) + cg];
                             const float4 h1 = hrow[rr * (DH / 4) + CG + cg];
                             const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-                            for (int i = 0; i < kVPT; ++i)
+                            for (int i = 0; i < kVPH; ++i)
 #pragma unroll
                                 for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(pv[i], hv[j], acc[i][j]);
                         }
@@ -308,8 +315,9 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             if (act) {
                 float *dst0 = part + (size_t)cr * kNSMax * E1;
 #pragma unroll
-                for (int i = 0; i < kVPT; ++i) {
-                    const int x = kVPT * vg + i;
+                for (int i = 0; i < kVPH; ++i) {
+                    if (i >= nvt) break;
+                    const int x = nvt * vg + i;
                     if (x >= nsc) break;
                     float *dst = dst0 + (size_t)x * E1;
                     if (hthr) {
@@ -488,40 +496,69 @@ lola_fused_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
             *reinterpret_cast<float4 *>(vm + mm * DH + a0 + 4) = make_float4(x[4], x[5], x[6], x[7]);
         }
         __syncthreads();
-        for (int rr = tid; nm > 0 && rr < nrows; rr += kFT) {  // one pass: R <= kFT
-            const int e = tab[rr];
-            const int a = e & 255, b = (e >> 8) & 255;
-            const float wgt = (e >> 16) ? kSqrt2 : 1.f;
-            float acc[DH];
+        // H[r] += sum_m phi_r(k_m) v_m, s[r] += sum_m phi_r(k_m): each thread a tile
+        // of RT rows x 16 columns (the pairs in list order, as one row at a time
+        // would add them), so a merged value read from shared memory feeds RT
+        // multiply-adds
+        {
+            constexpr int NCG = DH / 16, RT = DH / 16;  // column groups, rows per thread
+            const int cg = tid % NCG, rg = tid / NCG;
+            if (nm > 0 && RT * rg < nrows) {
+                int ea[RT], eb[RT];
+                float wgt[RT];
 #pragma unroll
-            for (int c = 0; c < DH; ++c) acc[c] = 0.f;
-            float sacc = 0.f;
-#pragma unroll 2
-            for (int mm = 0; mm < nm; ++mm) {
-                const int col = W + cand_key(mlist[mm]);
-                const float p = xv(XT + a * P + col) * xv(XT + b * P + col) * wgt;
-                const float4 *vr = reinterpret_cast<const float4 *>(vm + mm * DH);
-#pragma unroll
-                for (int c = 0; c < DH / 4; ++c) {
-                    const float4 x = vr[c];
-                    acc[4 * c] = fmaf(p, x.x, acc[4 * c]);
-                    acc[4 * c + 1] = fmaf(p, x.y, acc[4 * c + 1]);
-                    acc[4 * c + 2] = fmaf(p, x.z, acc[4 * c + 2]);
-                    acc[4 * c + 3] = fmaf(p, x.w, acc[4 * c + 3]);
+                for (int i = 0; i < RT; ++i) {
+                    const int e = RT * rg + i < nrows ? tab[RT * rg + i] : 0;
+                    ea[i] = e & 255;
+                    eb[i] = (e >> 8) & 255;
+                    wgt[i] = (e >> 16) ? kSqrt2 : 1.f;
                 }
-                sacc += p;
-            }
-            float4 *hr = reinterpret_cast<float4 *>(Hs + rr * DH);
+                float acc[RT][16], sacc[RT];
 #pragma unroll
-            for (int c = 0; c < DH / 4; ++c) {
-                float4 h = hr[c];
-                h.x += acc[4 * c];
-                h.y += acc[4 * c + 1];
-                h.z += acc[4 * c + 2];
-                h.w += acc[4 * c + 3];
-                hr[c] = h;
+                for (int i = 0; i < RT; ++i) {
+                    sacc[i] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) acc[i][c] = 0.f;
+                }
+#pragma unroll 2
+                for (int mm = 0; mm < nm; ++mm) {
+                    const int col = W + cand_key(mlist[mm]);
+                    float pv[RT];
+#pragma unroll
+                    for (int i = 0; i < RT; ++i)
+                        pv[i] = xv(XT + ea[i] * P + col) * xv(XT + eb[i] * P + col) * wgt[i];
+                    const float4 *vr = reinterpret_cast<const float4 *>(vm + mm * DH + 16 * cg);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float4 x = vr[c];
+#pragma unroll
+                        for (int i = 0; i < RT; ++i) {
+                            acc[i][4 * c] = fmaf(pv[i], x.x, acc[i][4 * c]);
+                            acc[i][4 * c + 1] = fmaf(pv[i], x.y, acc[i][4 * c + 1]);
+                            acc[i][4 * c + 2] = fmaf(pv[i], x.z, acc[i][4 * c + 2]);
+                            acc[i][4 * c + 3] = fmaf(pv[i], x.w, acc[i][4 * c + 3]);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < RT; ++i) sacc[i] += pv[i];
+                }
+#pragma unroll
+                for (int i = 0; i < RT; ++i) {
+                    const int rr = RT * rg + i;
+                    if (rr >= nrows) break;
+                    float4 *hr = reinterpret_cast<float4 *>(Hs + rr * DH + 16 * cg);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float4 h = hr[c];
+                        h.x += acc[i][4 * c];
+                        h.y += acc[i][4 * c + 1];
+                        h.z += acc[i][4 * c + 2];
+                        h.w += acc[i][4 * c + 3];
+                        hr[c] = h;
+                    }
+                    if (cg == 0) ss[rr] += sacc[i];
+                }
             }
-            ss[rr] += sacc;
         }
         // kept candidate n (of this CTA's share): phi(k)^T [H | s] after the merge
         {
