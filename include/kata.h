@@ -209,9 +209,17 @@ KATA_API size_t kata_prefill_host_workspace_bytes(int B, int H, int T, int d, in
 
 /*
  * kata_prefill with host inputs and output: copies q_host, k_host, v_host to
- * device staging inside `workspace`, runs kata_prefill on `stream` from a
- * zero state, and copies o back to o_host (all asynchronous on `stream`;
- * the caller synchronises before reading o_host).
+ * device staging inside `workspace`, runs kata_prefill from a zero state, and
+ * copies o back to o_host. The heads are processed in two pieces of
+ * consecutive heads (each head is independent), one on `stream` and one on a
+ * second stream the library keeps per device, so the host-to-device
+ * copies of one piece overlap the kernels and the device-to-host copy of
+ * another; `stream` is made to wait for the second stream before the call
+ * returns. Everything is asynchronous with respect to the host: the caller
+ * synchronises `stream` before reading o_host, and pinned host buffers are
+ * needed for the copies to overlap. The result equals kata_prefill's on the
+ * same inputs (the same kernels per head; the chunked form may split a
+ * piece's sequence differently, which changes fp32 rounding only).
  */
 KATA_API int kata_prefill_host(const void *q_host, const void *k_host, const void *v_host, int dtype,
                       int B, int H, int T, int d, int chunk, float eps, float *o_host,
